@@ -1,0 +1,153 @@
+/*
+ * lr_linear.h — C ABI of the B200 (sm_100a) low-rank linear layer library.
+ *
+ * The layer:   Y = (X · A) · B  (+ bias)
+ *
+ *   X    [M, K]  activations (M tokens)
+ *   A    [K, r]  first factor      } W [K, N] ≈ A · B, the factorisation that
+ *   B    [r, N]  second factor     } SVD-style compression puts in place of a
+ *   bias [N]     optional          } dense Y = X · W
+ *   Y    [M, N]  output
+ *
+ * Sources: "Why Smaller Is Slower? Dimensional Misalignment in Compressed
+ * LLMs" (GAC), §1 Introduction and Figure 1 — low-rank factorisation replaces
+ * W by A·B and makes the reduced rank r the inner dimension of two smaller
+ * GEMMs; LowRankArena review, "What SVD-based LLM compression actually does" —
+ * a truncated SVD stored as two factors, k(m+n) parameters, forward pass as
+ * two multiplies.  r is often not a multiple of 8 (e.g. 107, 1741); every
+ * entry point accepts any r >= 0.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are bf16 (IEEE bfloat16 bit patterns), row-major and
+ *     contiguous unless a leading dimension is given.  Accumulation is fp32;
+ *     Y is rounded once to bf16 (nearest-even) after the bias is added.
+ *   - Device pointers point to memory of the current CUDA device.  Any
+ *     2-byte-aligned pointer is accepted; 16-byte-aligned pointers with row
+ *     strides that are multiples of 8 elements take the TMA fast path.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: Y is valid once the stream has been synchronised.
+ *   - The caller owns every tensor.  The library owns a workspace per
+ *     (device, stream) for the intermediate T = X·A and split-K partial sums,
+ *     grown on demand with cudaMalloc (which synchronises the device); it is
+ *     kept until lr_release_workspaces() or process exit.
+ *   - Errors: invalid arguments return LR_ERR_INVALID_ARG before anything is
+ *     launched; a failed CUDA call returns LR_ERR_CUDA (see lr_last_cuda_error).
+ *     Device-side bounded waits that run out set a device status word, which
+ *     lr_last_device_status() reports; no kernel traps or asserts.
+ *   - Calls on one stream are ordered; calls that share a stream must not run
+ *     concurrently from several host threads.
+ */
+#ifndef LR_LINEAR_H
+#define LR_LINEAR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LR_OK = 0,
+  LR_ERR_INVALID_ARG = 1,  /* bad size, null or overlapping pointer            */
+  LR_ERR_UNSUPPORTED = 2,  /* no sm_100 device, or a size beyond int32 tiles  */
+  LR_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                */
+  LR_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out               */
+  LR_ERR_NO_MEMORY = 5     /* workspace allocation failed                      */
+} lr_status;
+
+/*
+ * lr_linear — Y = (X·A)·B + bias on the device.
+ *
+ * X [M,K], A [K,r], B [r,N], bias [N] (may be NULL), Y [M,N]: device
+ * pointers, bf16, row-major contiguous.  Y must not overlap X, A, B or bias.
+ * Sizes: 0 <= M, K, r, N < 2^31.  M == 0 or N == 0: nothing is launched.
+ * K == 0 or r == 0: the sum is empty and Y = bias (or 0).
+ *
+ * Path: M <= 16 takes the decode kernels (bandwidth-bound streaming of A then
+ * B, T kept in fp32); larger M takes the tcgen05 prefill kernels (T = X·A
+ * written once as bf16, then Y = T·B).  Neither path pads r on the host.
+ */
+lr_status lr_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                    int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
+
+/*
+ * One projection of a group (a decoder layer's q/k/v/o/gate/up/down).
+ * X [M,K] (entries may share one X pointer), A [K,r], B [r,N], bias [N] or
+ * NULL, Y with row stride ld_y >= N (so two projections can write the two
+ * halves of one packed [M, N1+N2] buffer, e.g. gate and up).
+ */
+typedef struct {
+  const void* X;
+  int64_t K;
+  const void* A;
+  const void* B;
+  const void* bias;
+  void* Y;
+  int64_t ld_y;
+  int64_t r;
+  int64_t N;
+} lr_proj;
+
+/*
+ * lr_linear_group — every projection of `projs` (n_proj >= 0) on the same M,
+ * in one call, on `stream`.  Each projection's result equals lr_linear on its
+ * own arguments.  The Y ranges (rows × [0, N) at stride ld_y) of different
+ * projections must not overlap each other or any input.  FlashSVD v1.5's
+ * abstract describes the packed execution of a layer's projections this
+ * mirrors (catalogue record of arXiv 2605.08314).
+ */
+lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream);
+
+/*
+ * lr_linear_host — the same layer on HOST buffers: copies X, A, B and bias
+ * to library-owned device buffers, runs lr_linear, copies Y back and
+ * synchronises `stream`.  Pinned host memory gives asynchronous copies;
+ * pageable memory works too.  Returns when Y (host) is written.
+ */
+lr_status lr_linear_host(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                         int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
+
+/*
+ * lr_dense — Y = X·W + bias, W [K,N], with the same kernels (the dense layer
+ * the factorisation replaces; the comparison the GAC paper's title asks
+ * about: is the smaller layer still slower?).
+ */
+lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int64_t M, int64_t K,
+                   int64_t N, void* stream);
+
+/*
+ * lr_last_device_status — synchronises `stream`, then reports and clears the
+ * device status word of the current device: LR_ERR_TIMEOUT if a bounded
+ * device-side wait ran out since the last call, else LR_OK.  After a timeout
+ * the kernels of later calls stop early until this is called.
+ */
+lr_status lr_last_device_status(void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* lr_status_string(lr_status s);
+
+/* The last CUDA error code (cudaError_t as int) seen by this thread. */
+int lr_last_cuda_error(void);
+
+/*
+ * lr_set_path — testing and benchmarking control of the dispatch:
+ *   0 = automatic (M <= 16 decode, else prefill), 1 = force decode (M <= 16
+ *   only; larger M returns LR_ERR_INVALID_ARG), 2 = force prefill.
+ * lr_set_wait_limit_ns — time limit of every device-side bounded wait
+ *   (default 2e9 ns); 0 restores the default.
+ * Both are process-wide and take effect on the next call.
+ */
+lr_status lr_set_path(int path);
+lr_status lr_set_wait_limit_ns(int64_t ns);
+
+/* Counts the kernels launched by this library in this process. */
+int64_t lr_kernel_launch_count(void);
+
+/* Frees every workspace and staging buffer (synchronises each device). */
+lr_status lr_release_workspaces(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LR_LINEAR_H */

@@ -1,0 +1,214 @@
+"""rank_linear_layers_b200 — B200 (sm_100a) low-rank linear layer Y = (X·A)·B (+bias).
+
+A thin ctypes binding over ``liblrlinear.so`` (C ABI in ``include/lr_linear.h``).
+This module only marshals arguments: torch tensors supply device pointers and
+the current CUDA stream; every step of the layer runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback: if the library is missing or
+was built for another GPU, calls raise.
+
+    import torch, rank_linear_layers_b200 as lr
+    Y = lr.lr_linear(X, A, B)            # X [M,K], A [K,r], B [r,N] bf16 cuda
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblrlinear.so")
+
+LR_OK = 0
+LR_ERR_INVALID_ARG = 1
+LR_ERR_UNSUPPORTED = 2
+LR_ERR_CUDA = 3
+LR_ERR_TIMEOUT = 4
+LR_ERR_NO_MEMORY = 5
+
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+
+# Every symbol include/lr_linear.h declares.
+EXPORTS = (
+    "lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense", "lr_last_device_status",
+    "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
+    "lr_kernel_launch_count", "lr_release_workspaces",
+)
+
+
+class LrError(RuntimeError):
+    def __init__(self, code: int, what: str, cuda_error: int = 0):
+        self.code = code
+        self.cuda_error = cuda_error
+        super().__init__(f"{what}: {status_string(code)} (cuda error {cuda_error})")
+
+
+class LrProj(ctypes.Structure):
+    _fields_ = [
+        ("X", ctypes.c_void_p), ("K", ctypes.c_int64), ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+        ("ld_y", ctypes.c_int64), ("r", ctypes.c_int64), ("N", ctypes.c_int64),
+    ]
+
+
+_lib = None
+
+
+def lib(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m rank_linear_layers_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(path)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    L.lr_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    L.lr_linear_group.argtypes = [ctypes.POINTER(LrProj), ctypes.c_int, i64, vp]
+    L.lr_linear_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    L.lr_dense.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+    L.lr_last_device_status.argtypes = [vp]
+    L.lr_status_string.argtypes = [ctypes.c_int]
+    L.lr_status_string.restype = ctypes.c_char_p
+    L.lr_last_cuda_error.argtypes = []
+    L.lr_set_path.argtypes = [ctypes.c_int]
+    L.lr_set_wait_limit_ns.argtypes = [i64]
+    L.lr_kernel_launch_count.argtypes = []
+    L.lr_kernel_launch_count.restype = i64
+    L.lr_release_workspaces.argtypes = []
+    for name in ("lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense",
+                 "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
+                 "lr_set_wait_limit_ns", "lr_release_workspaces"):
+        getattr(L, name).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().lr_status_string(code).decode()
+    except Exception:
+        return f"status {code}"
+
+
+def _check(code: int, what: str):
+    if code != LR_OK:
+        raise LrError(code, what, lib().lr_last_cuda_error())
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_bf16(name, t, shape=None):
+    import torch
+    if t is None:
+        return
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a bf16 CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def lr_linear(X, A, B, bias=None, Y=None, stream=None):
+    """Y = (X·A)·B + bias on the GPU (bf16 in/out, fp32 accumulation)."""
+    import torch
+    M, K = X.shape
+    r = A.shape[1]
+    N = B.shape[1]
+    _check_bf16("X", X)
+    _check_bf16("A", A, (K, r))
+    _check_bf16("B", B, (r, N))
+    _check_bf16("bias", bias, (N,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _check_bf16("Y", Y, (M, N))
+    _check(lib().lr_linear(_ptr(X), _ptr(A), _ptr(B), _ptr(bias), _ptr(Y), M, K, r, N,
+                           _stream_ptr(stream)), "lr_linear")
+    return Y
+
+
+def lr_dense(X, W, bias=None, Y=None, stream=None):
+    """Y = X·W + bias with the same kernels (the dense comparison)."""
+    import torch
+    M, K = X.shape
+    N = W.shape[1]
+    _check_bf16("X", X)
+    _check_bf16("W", W, (K, N))
+    _check_bf16("bias", bias, (N,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _check_bf16("Y", Y, (M, N))
+    _check(lib().lr_dense(_ptr(X), _ptr(W), _ptr(bias), _ptr(Y), M, K, N, _stream_ptr(stream)),
+           "lr_dense")
+    return Y
+
+
+def lr_linear_group(projs: Sequence[dict], M: int, stream=None):
+    """Run several projections on the same M in one call.
+
+    Each dict has X, A, B, Y (torch tensors or raw pointer ints), and
+    optionally bias, ld_y (default N), K, r, N (taken from shapes when the
+    entries are tensors).  Y may be a view into a packed buffer: pass the
+    element pointer and ld_y explicitly via ``Y_ptr`` / ``ld_y``.
+    """
+    arr = (LrProj * max(1, len(projs)))()
+    for i, p in enumerate(projs):
+        A, B = p["A"], p["B"]
+        K = p.get("K", A.shape[0] if hasattr(A, "shape") else None)
+        r = p.get("r", A.shape[1] if hasattr(A, "shape") else None)
+        N = p.get("N", B.shape[1] if hasattr(B, "shape") else None)
+        y_ptr = p.get("Y_ptr", _ptr(p.get("Y")))
+        arr[i] = LrProj(_ptr(p["X"]) if hasattr(p["X"], "data_ptr") else p["X"], K,
+                        _ptr(A) if hasattr(A, "data_ptr") else A,
+                        _ptr(B) if hasattr(B, "data_ptr") else B,
+                        _ptr(p.get("bias")) if hasattr(p.get("bias"), "data_ptr") else p.get("bias"),
+                        y_ptr, p.get("ld_y", N), r, N)
+    _check(lib().lr_linear_group(arr, len(projs), M, _stream_ptr(stream)), "lr_linear_group")
+
+
+def lr_linear_host(X, A, B, bias=None, Y=None, stream=None):
+    """The layer on HOST tensors (pinned or pageable): copies in, computes, copies out."""
+    import torch
+    M, K = X.shape
+    r = A.shape[1]
+    N = B.shape[1]
+    for name, t in (("X", X), ("A", A), ("B", B), ("bias", bias)):
+        if t is not None and (t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous bf16 host tensor")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=X.is_pinned())
+    _check(lib().lr_linear_host(_ptr(X), _ptr(A), _ptr(B), _ptr(bias), _ptr(Y), M, K, r, N,
+                                _stream_ptr(stream)), "lr_linear_host")
+    return Y
+
+
+def last_device_status(stream=None) -> int:
+    return lib().lr_last_device_status(_stream_ptr(stream))
+
+
+def set_path(path: int):
+    _check(lib().lr_set_path(path), "lr_set_path")
+
+
+def set_wait_limit_ns(ns: int):
+    _check(lib().lr_set_wait_limit_ns(ns), "lr_set_wait_limit_ns")
+
+
+def kernel_launch_count() -> int:
+    return int(lib().lr_kernel_launch_count())
+
+
+def release_workspaces():
+    _check(lib().lr_release_workspaces(), "lr_release_workspaces")

@@ -1,0 +1,561 @@
+// lr_api.cu — the C ABI of include/lr_linear.h: argument validation, path
+// selection, workspaces, TMA descriptors and status reporting.  Every step
+// of the layer itself runs in the kernels of lr_decode.cu and lr_umma.cu.
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <set>
+#include <tuple>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/lr_linear.h"
+#include "lr_internal.h"
+
+namespace lr {
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<int> g_path{0};
+std::atomic<long long> g_wait_ns{0};
+std::atomic<long long> g_launches{0};
+constexpr long long kDefaultWaitNs = 2000000000LL;
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  DevStatus* status = nullptr;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+
+struct Workspace {
+  char* ptr = nullptr;
+  size_t cap = 0;
+  size_t zero_bytes = 0;  // prefix that is all-zero between calls
+};
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+struct Staging {
+  char* ptr = nullptr;
+  size_t cap = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Staging> g_stage;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+struct MapKey {
+  const void* ptr;
+  uint64_t inner, outer, stride;
+  uint32_t box_inner, box_outer;
+  bool operator<(const MapKey& o) const {
+    return std::tie(ptr, inner, outer, stride, box_inner, box_outer) <
+           std::tie(o.ptr, o.inner, o.outer, o.stride, o.box_inner, o.box_outer);
+  }
+};
+std::map<MapKey, CUtensorMap> g_maps;
+
+lr_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  if (e == cudaErrorMemoryAllocation) return LR_ERR_NO_MEMORY;
+  return LR_ERR_CUDA;
+}
+
+#define LR_CUDA(call)                          \
+  do {                                         \
+    cudaError_t e_ = (call);                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+lr_status device_info(DeviceInfo** out, int* dev_out) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) {
+    DeviceInfo d;
+    LR_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    LR_CUDA(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev));
+    if (d.major != 10) return LR_ERR_UNSUPPORTED;
+    LR_CUDA(cudaMalloc(&d.status, sizeof(DevStatus)));
+    LR_CUDA(cudaMemset(d.status, 0, sizeof(DevStatus)));
+    it = g_dev.emplace(dev, d).first;
+  }
+  *out = &it->second;
+  *dev_out = dev;
+  return LR_OK;
+}
+
+lr_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return LR_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  LR_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+  if (q != cudaDriverEntryPointSuccess || fn == nullptr) return LR_ERR_UNSUPPORTED;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return LR_OK;
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
+lr_status tensor_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
+                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer) {
+  lr_status st = get_encoder();
+  if (st != LR_OK) return st;
+  MapKey key{ptr, inner, outer, row_stride_elems, box_inner, box_outer};
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return LR_OK;
+    }
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return LR_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps.emplace(key, *out);
+  return LR_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// A workspace whose first `zero_need` bytes are zero on entry (and must be
+// left zero by the kernels) followed by `scratch_need` bytes of scratch.
+lr_status workspace(cudaStream_t stream, size_t zero_need, size_t scratch_need, char** zero,
+                    char** scratch) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  zero_need = align_up(zero_need, 256);
+  const size_t z = std::max(zero_need, w.zero_bytes);
+  const size_t need = z + align_up(scratch_need, 256);
+  if (need > w.cap) {
+    if (w.ptr) {
+      LR_CUDA(cudaStreamSynchronize(stream));
+      LR_CUDA(cudaFree(w.ptr));
+      w.ptr = nullptr;
+      w.cap = 0;
+    }
+    const size_t cap = align_up(need + need / 4, 1 << 20);
+    LR_CUDA(cudaMalloc(&w.ptr, cap));
+    w.cap = cap;
+    LR_CUDA(cudaMemsetAsync(w.ptr, 0, z, stream));
+    w.zero_bytes = z;
+  } else if (z > w.zero_bytes) {
+    LR_CUDA(cudaMemsetAsync(w.ptr + w.zero_bytes, 0, z - w.zero_bytes, stream));
+    w.zero_bytes = z;
+  }
+  *zero = w.ptr;
+  *scratch = w.ptr + w.zero_bytes;
+  return LR_OK;
+}
+
+bool ranges_overlap(const void* a, size_t abytes, const void* b, size_t bbytes) {
+  if (!a || !b || abytes == 0 || bbytes == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bbytes && b0 < a0 + abytes;
+}
+
+size_t span_bytes(int64_t rows, int64_t cols, int64_t ld) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return static_cast<size_t>((rows - 1) * ld + cols) * 2;
+}
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
+
+WaitCtl wait_ctl(DeviceInfo* d) {
+  long long ns = g_wait_ns.load();
+  return WaitCtl{d->status, static_cast<unsigned long long>(ns > 0 ? ns : kDefaultWaitNs)};
+}
+
+lr_status validate(const void* X, const void* A, const void* B, const void* bias, const void* Y,
+                   int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy) {
+  if (M < 0 || K < 0 || r < 0 || N < 0) return LR_ERR_INVALID_ARG;
+  if (M > kMaxDim || K > kMaxDim || r > kMaxDim || N > kMaxDim) return LR_ERR_UNSUPPORTED;
+  if (ldy < N) return LR_ERR_INVALID_ARG;
+  if (M > 0 && N > 0 && !Y) return LR_ERR_INVALID_ARG;
+  if (M > 0 && K > 0 && r > 0 && N > 0 && (!X || !A || !B)) return LR_ERR_INVALID_ARG;
+  for (const void* p : {X, A, B, bias, Y})
+    if (p && !aligned2(p)) return LR_ERR_INVALID_ARG;
+  const size_t ybytes = span_bytes(M, N, ldy);
+  if (ranges_overlap(Y, ybytes, X, span_bytes(M, K, K)) ||
+      ranges_overlap(Y, ybytes, A, span_bytes(K, r, r)) ||
+      ranges_overlap(Y, ybytes, B, span_bytes(r, N, N)) ||
+      ranges_overlap(Y, ybytes, bias, span_bytes(1, N, N)))
+    return LR_ERR_INVALID_ARG;
+  return LR_OK;
+}
+
+lr_status launched(cudaError_t e, int n = 1) {
+  if (e != cudaSuccess) return cuda_fail(e);
+  g_launches += n;
+  return LR_OK;
+}
+
+// out = V · W (+bias) for M <= 16 tokens through one skinny launch.
+lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64_t ldv, bool v_f32,
+                 const void* W, int64_t Kd, int64_t Nd, float* acc, unsigned int* counters,
+                 float* out_f32, int64_t ld_out_f32, void* out_bf16, int64_t ld_out,
+                 const void* bias) {
+  const SkinnyPlan plan = plan_skinny(M, Kd, Nd, d->sms);
+  SkinnyArgs a{};
+  a.M = M;
+  a.Kd = Kd;
+  a.Nd = Nd;
+  a.V = V;
+  a.ldv = ldv;
+  a.v_f32 = v_f32 ? 1 : 0;
+  a.W = static_cast<const __nv_bfloat16*>(W);
+  a.ldw = Nd;
+  a.w_lo = reinterpret_cast<uintptr_t>(W);
+  a.w_hi = a.w_lo + static_cast<uintptr_t>(Kd * Nd * 2);
+  a.acc = acc;
+  a.ld_acc = static_cast<int64_t>(align_up(static_cast<size_t>(Nd), 4));
+  a.counters = counters;
+  a.out_f32 = out_f32;
+  a.ld_out_f32 = ld_out_f32;
+  a.out_bf16 = static_cast<__nv_bfloat16*>(out_bf16);
+  a.ld_out = ld_out;
+  a.bias = static_cast<const __nv_bfloat16*>(bias);
+  return launched(launch_skinny(plan, a, stream));
+}
+
+size_t acc_bytes(int M, int64_t n) { return align_up(static_cast<size_t>(M) * align_up(n, 4) * 4, 256); }
+size_t ctr_bytes(int M, int64_t Kd, int64_t n, int sms) {
+  const SkinnyPlan p = plan_skinny(M, Kd, n, sms);
+  return align_up(static_cast<size_t>(p.col_blocks) * 4, 256);
+}
+
+lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
+                     const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
+                     int64_t N, int64_t ldy) {
+  const int m = static_cast<int>(M);
+  const size_t acc1 = acc_bytes(m, r), acc2 = acc_bytes(m, N);
+  const size_t c1 = ctr_bytes(m, K, r, d->sms), c2 = ctr_bytes(m, r, N, d->sms);
+  const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), 4));
+  char *zero = nullptr, *scratch = nullptr;
+  lr_status st = workspace(stream, acc1 + acc2 + c1 + c2, static_cast<size_t>(M) * ldt * 4, &zero,
+                           &scratch);
+  if (st != LR_OK) return st;
+  float* a1 = reinterpret_cast<float*>(zero);
+  float* a2 = reinterpret_cast<float*>(zero + acc1);
+  unsigned int* k1 = reinterpret_cast<unsigned int*>(zero + acc1 + acc2);
+  unsigned int* k2 = reinterpret_cast<unsigned int*>(zero + acc1 + acc2 + c1);
+  float* T = reinterpret_cast<float*>(scratch);
+  // Phase 1: T = X·A (fp32).  Phase 2: Y = T·B + bias.
+  st = skinny(d, stream, m, X, K, false, A, K, r, a1, k1, T, ldt, nullptr, 0, nullptr);
+  if (st != LR_OK) return st;
+  return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias);
+}
+
+lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, const void* b,
+               int64_t ldb, void* c, int64_t ldc, const void* bias, int64_t Mr, int64_t Nc,
+               int64_t Kc, size_t a_bytes, size_t b_bytes) {
+  GemmArgs g{};
+  g.Mr = static_cast<int>(Mr);
+  g.Nc = static_cast<int>(Nc);
+  g.Kc = static_cast<int>(Kc);
+  g.a = static_cast<const __nv_bfloat16*>(a);
+  g.lda = lda;
+  g.a_lo = reinterpret_cast<uintptr_t>(a);
+  g.a_hi = g.a_lo + a_bytes;
+  g.b = static_cast<const __nv_bfloat16*>(b);
+  g.ldb = ldb;
+  g.b_lo = reinterpret_cast<uintptr_t>(b);
+  g.b_hi = g.b_lo + b_bytes;
+  g.c = static_cast<__nv_bfloat16*>(c);
+  g.ldc = ldc;
+  g.bias = static_cast<const __nv_bfloat16*>(bias);
+  g.tiles_m = static_cast<int>((Mr + kGemmBM - 1) / kGemmBM);
+  g.tiles_n = static_cast<int>((Nc + kGemmBN - 1) / kGemmBN);
+  g.wait = wait_ctl(d);
+  GemmMaps maps{};
+  maps.a_tma = (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (lda % 8 == 0);
+  maps.b_tma = (reinterpret_cast<uintptr_t>(b) % 16 == 0) && (ldb % 8 == 0);
+  if (maps.a_tma) {
+    lr_status st = tensor_map(&maps.a, a, Kc, Mr, lda, kGemmBK, kGemmBM);
+    if (st != LR_OK) return st;
+  }
+  if (maps.b_tma) {
+    lr_status st = tensor_map(&maps.b, b, Nc, Kc, ldb, 64, kGemmBK);
+    if (st != LR_OK) return st;
+  }
+  return launched(launch_gemm(g, maps, d->sms, stream));
+}
+
+lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
+                      const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
+                      int64_t N, int64_t ldy) {
+  const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), 8));
+  char *zero = nullptr, *scratch = nullptr;
+  lr_status st = workspace(stream, 0, static_cast<size_t>(M) * ldt * 2, &zero, &scratch);
+  if (st != LR_OK) return st;
+  void* T = scratch;
+  st = gemm(d, stream, X, K, A, r, T, ldt, nullptr, M, r, K, span_bytes(M, K, K),
+            span_bytes(K, r, r));
+  if (st != LR_OK) return st;
+  return gemm(d, stream, T, ldt, B, N, Y, ldy, bias, M, N, r, span_bytes(M, r, ldt),
+              span_bytes(r, N, N));
+}
+
+lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                     int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, cudaStream_t stream) {
+  lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy);
+  if (st != LR_OK) return st;
+  const int path = g_path.load();
+  if (path == 1 && M > 16) return LR_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return LR_OK;
+  DeviceInfo* d = nullptr;
+  int dev = 0;
+  st = device_info(&d, &dev);
+  if (st != LR_OK) return st;
+  if (K == 0 || r == 0) return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), ldy, M, N,
+                                                         static_cast<const __nv_bfloat16*>(bias),
+                                                         stream));
+  const bool decode = (path == 1) || (path == 0 && M <= 16);
+  if (decode) return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+  return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+}
+
+
+// Two projections' outputs may interleave (gate and up writing the two halves
+// of one packed buffer) but must not share an element.  Conservative: equal
+// row strides and no row that spills into the next are required when the byte
+// ranges overlap at all.
+bool y_disjoint(const lr_proj& p, const lr_proj& q, int64_t M) {
+  if (!p.Y || !q.Y || M == 0 || p.N == 0 || q.N == 0) return true;
+  if (!ranges_overlap(p.Y, span_bytes(M, p.N, p.ld_y), q.Y, span_bytes(M, q.N, q.ld_y)))
+    return true;
+  if (p.ld_y != q.ld_y) return false;
+  const intptr_t d = reinterpret_cast<intptr_t>(q.Y) - reinterpret_cast<intptr_t>(p.Y);
+  if (d % 2 != 0) return false;
+  const int64_t off = d / 2, ld = p.ld_y;
+  int64_t a = off / ld, b = off % ld;
+  if (b < 0) {
+    b += ld;
+    a -= 1;
+  }
+  if (b + q.N > ld) return false;
+  const bool rows = (a < 0 ? -a : a) < M;
+  const bool cols = b < p.N;
+  return !(rows && cols);
+}
+
+}  // namespace
+
+cudaError_t ensure_max_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, int, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({kernel, dev, bytes})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({kernel, dev, bytes});
+  return e;
+}
+
+}  // namespace lr
+
+using namespace lr;
+
+extern "C" {
+
+lr_status lr_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                    int64_t M, int64_t K, int64_t r, int64_t N, void* stream) {
+  return run_linear(X, A, B, bias, Y, M, K, r, N, N, static_cast<cudaStream_t>(stream));
+}
+
+lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream) {
+  if (n_proj < 0 || (n_proj > 0 && !projs) || M < 0) return LR_ERR_INVALID_ARG;
+  // Validate everything before the first launch, including Y overlaps.
+  for (int i = 0; i < n_proj; ++i) {
+    const lr_proj& p = projs[i];
+    lr_status st = validate(p.X, p.A, p.B, p.bias, p.Y, M, p.K, p.r, p.N, p.ld_y);
+    if (st != LR_OK) return st;
+    const size_t yi = span_bytes(M, p.N, p.ld_y);
+    for (int j = 0; j < n_proj; ++j) {
+      const lr_proj& q = projs[j];
+      if (j != i) {
+        if (!y_disjoint(p, q, M)) return LR_ERR_INVALID_ARG;
+        if (ranges_overlap(p.Y, yi, q.X, span_bytes(M, q.K, q.K)) ||
+            ranges_overlap(p.Y, yi, q.A, span_bytes(q.K, q.r, q.r)) ||
+            ranges_overlap(p.Y, yi, q.B, span_bytes(q.r, q.N, q.N)) ||
+            ranges_overlap(p.Y, yi, q.bias, span_bytes(1, q.N, q.N)))
+          return LR_ERR_INVALID_ARG;
+      }
+    }
+  }
+  for (int i = 0; i < n_proj; ++i) {
+    const lr_proj& p = projs[i];
+    lr_status st = run_linear(p.X, p.A, p.B, p.bias, p.Y, M, p.K, p.r, p.N, p.ld_y,
+                              static_cast<cudaStream_t>(stream));
+    if (st != LR_OK) return st;
+  }
+  return LR_OK;
+}
+
+lr_status lr_linear_host(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                         int64_t M, int64_t K, int64_t r, int64_t N, void* stream_) {
+  if (M < 0 || K < 0 || r < 0 || N < 0) return LR_ERR_INVALID_ARG;
+  if (M > kMaxDim || K > kMaxDim || r > kMaxDim || N > kMaxDim) return LR_ERR_UNSUPPORTED;
+  if (M > 0 && N > 0 && !Y) return LR_ERR_INVALID_ARG;
+  if (M > 0 && K > 0 && r > 0 && N > 0 && (!X || !A || !B)) return LR_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return LR_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const size_t bx = align_up(static_cast<size_t>(M * K) * 2, 256);
+  const size_t ba = align_up(static_cast<size_t>(K * r) * 2, 256);
+  const size_t bb = align_up(static_cast<size_t>(r * N) * 2, 256);
+  const size_t bz = align_up(static_cast<size_t>(N) * 2, 256);
+  const size_t by = align_up(static_cast<size_t>(M * N) * 2, 256);
+  const size_t need = bx + ba + bb + bz + by;
+  char* base = nullptr;
+  {
+    int dev = 0;
+    LR_CUDA(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(g_mu);
+    Staging& s = g_stage[{dev, stream}];
+    if (need > s.cap) {
+      if (s.ptr) {
+        LR_CUDA(cudaStreamSynchronize(stream));
+        LR_CUDA(cudaFree(s.ptr));
+        s.ptr = nullptr;
+        s.cap = 0;
+      }
+      LR_CUDA(cudaMalloc(&s.ptr, need));
+      s.cap = need;
+    }
+    base = s.ptr;
+  }
+  char* dX = base;
+  char* dA = dX + bx;
+  char* dB = dA + ba;
+  char* dz = dB + bb;
+  char* dY = dz + bz;
+  if (M * K) LR_CUDA(cudaMemcpyAsync(dX, X, M * K * 2, cudaMemcpyHostToDevice, stream));
+  if (K * r) LR_CUDA(cudaMemcpyAsync(dA, A, K * r * 2, cudaMemcpyHostToDevice, stream));
+  if (r * N) LR_CUDA(cudaMemcpyAsync(dB, B, r * N * 2, cudaMemcpyHostToDevice, stream));
+  if (bias) LR_CUDA(cudaMemcpyAsync(dz, bias, N * 2, cudaMemcpyHostToDevice, stream));
+  lr_status st = run_linear(dX, dA, dB, bias ? dz : nullptr, dY, M, K, r, N, N, stream);
+  if (st != LR_OK) return st;
+  LR_CUDA(cudaMemcpyAsync(Y, dY, M * N * 2, cudaMemcpyDeviceToHost, stream));
+  LR_CUDA(cudaStreamSynchronize(stream));
+  return LR_OK;
+}
+
+lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int64_t M, int64_t K,
+                   int64_t N, void* stream_) {
+  // W [K, N] plays the role of A with r = N (no second factor).
+  lr_status st = validate(X, W, W, bias, Y, M, K, N, N, N);
+  if (st != LR_OK) return st;
+  if (M == 0 || N == 0) return LR_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DeviceInfo* d = nullptr;
+  int dev = 0;
+  st = device_info(&d, &dev);
+  if (st != LR_OK) return st;
+  if (K == 0)
+    return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), N, M, N,
+                                     static_cast<const __nv_bfloat16*>(bias), stream));
+  const int path = g_path.load();
+  const bool decode = (path == 1) || (path == 0 && M <= 16);
+  if (decode) {
+    if (M > 16) return LR_ERR_INVALID_ARG;
+    const int m = static_cast<int>(M);
+    const size_t acc = acc_bytes(m, N), c = ctr_bytes(m, K, N, d->sms);
+    char *zero = nullptr, *scratch = nullptr;
+    st = workspace(stream, acc + c, 0, &zero, &scratch);
+    if (st != LR_OK) return st;
+    return skinny(d, stream, m, X, K, false, W, K, N, reinterpret_cast<float*>(zero),
+                  reinterpret_cast<unsigned int*>(zero + acc), nullptr, 0, Y, N, bias);
+  }
+  return gemm(d, stream, X, K, W, N, Y, N, bias, M, N, K, span_bytes(M, K, K),
+              span_bytes(K, N, N));
+}
+
+lr_status lr_last_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  DeviceInfo* d = nullptr;
+  int dev = 0;
+  lr_status st = device_info(&d, &dev);
+  if (st != LR_OK) return st;
+  DevStatus h{};
+  LR_CUDA(cudaMemcpy(&h, d->status, sizeof h, cudaMemcpyDeviceToHost));
+  if (h.code == 0 && h.abort == 0) return LR_OK;
+  LR_CUDA(cudaMemset(d->status, 0, sizeof(DevStatus)));
+  return (h.code & LR_DEV_TIMEOUT) ? LR_ERR_TIMEOUT : LR_ERR_CUDA;
+}
+
+const char* lr_status_string(lr_status s) {
+  switch (s) {
+    case LR_OK: return "LR_OK";
+    case LR_ERR_INVALID_ARG: return "LR_ERR_INVALID_ARG";
+    case LR_ERR_UNSUPPORTED: return "LR_ERR_UNSUPPORTED";
+    case LR_ERR_CUDA: return "LR_ERR_CUDA";
+    case LR_ERR_TIMEOUT: return "LR_ERR_TIMEOUT";
+    case LR_ERR_NO_MEMORY: return "LR_ERR_NO_MEMORY";
+  }
+  return "LR_ERR_UNKNOWN";
+}
+
+int lr_last_cuda_error(void) { return g_last_cuda_error; }
+
+lr_status lr_set_path(int path) {
+  if (path < 0 || path > 2) return LR_ERR_INVALID_ARG;
+  g_path.store(path);
+  return LR_OK;
+}
+
+lr_status lr_set_wait_limit_ns(int64_t ns) {
+  if (ns < 0) return LR_ERR_INVALID_ARG;
+  g_wait_ns.store(ns);
+  return LR_OK;
+}
+
+int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
+
+lr_status lr_release_workspaces(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_ws) {
+    if (!kv.second.ptr) continue;
+    cudaSetDevice(kv.first.first);
+    cudaStreamSynchronize(kv.first.second);
+    cudaFree(kv.second.ptr);
+  }
+  g_ws.clear();
+  for (auto& kv : g_stage) {
+    if (!kv.second.ptr) continue;
+    cudaSetDevice(kv.first.first);
+    cudaStreamSynchronize(kv.first.second);
+    cudaFree(kv.second.ptr);
+  }
+  g_stage.clear();
+  g_maps.clear();
+  cudaSetDevice(cur);
+  return LR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// lr_internal.h — declarations shared by the host library and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "lr_ptx.cuh"
+
+namespace lr {
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
+cudaError_t ensure_max_smem(const void* kernel, int bytes);
+
+// ------------------------------------------------------------------ decode
+// out[m, n] = sum_k V[m, k] · W[k, n] for m < M (M <= 16), W a bf16 [Kd, Nd]
+// row-major matrix with row stride ldw.  Split over column blocks (grid.x)
+// and row ranges of W (grid.y); partial sums go to acc with fp32 atomics and
+// the last CTA of each column block writes the result and re-zeroes acc and
+// its counter, so the workspace is zero again when the launch ends.
+struct SkinnyArgs {
+  int M;
+  int64_t Kd, Nd;
+  const void* V;   // [M, ldv], bf16 (v_f32 == 0) or fp32
+  int64_t ldv;
+  int v_f32;
+  const __nv_bfloat16* W;
+  int64_t ldw;
+  uintptr_t w_lo, w_hi;  // byte extent of W's buffer
+  float* acc;            // [M, ld_acc] fp32, zero at rest
+  int64_t ld_acc;
+  unsigned int* counters;  // one per column block, zero at rest
+  int k_chunk;             // rows of W per CTA
+  int splits;              // == gridDim.y
+  float* out_f32;          // if non-null: fp32 result [M, ld_out_f32]
+  int64_t ld_out_f32;
+  __nv_bfloat16* out_bf16;  // else bf16 result (+bias) [M, ld_out]
+  int64_t ld_out;
+  const __nv_bfloat16* bias;
+};
+
+enum class SkinnyKind { kFma, kMma };
+
+struct SkinnyPlan {
+  SkinnyKind kind;
+  int mt;         // token tile (1, 2, 4 or 16)
+  int cols;       // columns per CTA
+  int threads;    // threads per CTA
+  int k_chunk;
+  int splits;
+  int col_blocks;
+  size_t smem;    // dynamic shared memory bytes
+};
+
+SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms);
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& args, cudaStream_t stream);
+
+// ------------------------------------------------------------------ prefill
+// C[Mr, Nc] = Aop[Mr, Kc] · Bop[Kc, Nc] (+ bias), bf16 in, fp32 accumulate,
+// bf16 out.  Aop is row-major (K contiguous), Bop is row-major (N contiguous).
+struct GemmArgs {
+  int Mr, Nc, Kc;
+  const __nv_bfloat16* a;
+  int64_t lda;
+  uintptr_t a_lo, a_hi;
+  const __nv_bfloat16* b;
+  int64_t ldb;
+  uintptr_t b_lo, b_hi;
+  __nv_bfloat16* c;
+  int64_t ldc;
+  const __nv_bfloat16* bias;
+  int tiles_m, tiles_n;
+  WaitCtl wait;
+};
+
+struct GemmMaps {
+  CUtensorMap a;  // valid when a_tma
+  CUtensorMap b;  // valid when b_tma
+  bool a_tma, b_tma;
+};
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;
+constexpr int kGemmStages = 4;
+
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(const GemmArgs& args, const GemmMaps& maps, int num_sms,
+                        cudaStream_t stream);
+
+// Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0).
+cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+                             const __nv_bfloat16* bias, cudaStream_t stream);
+
+}  // namespace lr

@@ -1,0 +1,396 @@
+// lr_umma.cu — tcgen05 (5th-generation tensor core) GEMM tile engine for the
+// prefill path of Y = (X·A)·B (+bias).
+//
+//   GEMM1:  T [M, r] = X [M, K] · A [K, r]        (T written once, bf16)
+//   GEMM2:  Y [M, N] = T [M, r] · B [r, N] + bias
+//
+// Both are C = Aop · Bop with Aop row-major (K contiguous: "K-major") and
+// Bop row-major (N contiguous: "MN-major"); the tensor core reads both
+// layouts from shared memory directly, so no operand is transposed.
+//
+// Structure (one persistent CTA per SM, warp-specialised):
+//   warps 0-3  epilogue: TMEM -> registers -> +bias -> bf16 -> global
+//   warp 4     one elected thread issues tcgen05.mma (128×256×16 per issue)
+//   warp 5     one thread issues TMA tile loads for operands whose row
+//              stride is a multiple of 16 bytes (TMA's requirement)
+//   warps 6-9  (only when an operand's row stride is not a multiple of 16
+//              bytes, e.g. A [K, r] with odd r) realigning loaders that write
+//              the same 128-byte-swizzled layout TMA would
+// A 4-stage shared-memory ring (mbarrier full/empty pairs) feeds the MMA;
+// two TMEM accumulators (2 × 256 fp32 columns) let the epilogue of one tile
+// overlap the main loop of the next.
+//
+// Ragged edges cost no padding on the host: TMA zero-fills out-of-bounds
+// rows and columns, the loaders zero them, the last K block issues only the
+// 16-deep MMA steps it needs, and the epilogue predicates rows and columns.
+// This is the point of the GAC paper's §3 analysis (misaligned K or N fall to
+// slower library kernels and partially filled tensor-core tiles): here a
+// misaligned r changes the loader, not the tile shape or the MMA rate.
+#include <algorithm>
+
+#include "lr_internal.h"
+#include "lr_load.cuh"
+
+namespace lr {
+
+namespace {
+
+constexpr int BM = kGemmBM;
+constexpr int BN = kGemmBN;
+constexpr int BK = kGemmBK;
+constexpr int STAGES = kGemmStages;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KB
+constexpr int B_STAGE = BK * BN * 2;  // 32 KB
+constexpr int STAGE = A_STAGE + B_STAGE;
+constexpr int B_ATOM = BK * 128;      // one 64-column MN-major atom column: 8 KB
+constexpr int EPI_WARPS = 4;
+constexpr int MMA_WARP = 4;
+constexpr int TMA_WARP = 5;
+constexpr int LOADER_WARP0 = 6;
+constexpr int LOADER_WARPS = 4;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+
+constexpr unsigned kWhereProducer = 1, kWhereLoader = 2, kWhereMma = 3, kWhereMmaAcc = 4,
+                   kWhereEpilogue = 5;
+
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                unsigned long long limit_ns) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+struct Smem {
+  uint8_t* base;  // 1024-aligned
+  __device__ uint8_t* a(int s) const { return base + s * STAGE; }
+  __device__ uint8_t* b(int s) const { return base + s * STAGE + A_STAGE; }
+};
+
+// Manual (realigning) load of Aop's [128 × 64] K-major tile for k block kb.
+// Each loader warp fills 32 rows, four rows (8 lanes each) per instruction.
+__device__ __forceinline__ void load_a_manual(uint8_t* dst, const GemmArgs& g, int m_blk, int kb,
+                                              int lw, int lane) {
+  const int gl = lane & 7;
+  const int k0 = kb * BK;
+  const int kvalid = min(BK, g.Kc - k0);
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = lw * 32 + 4 * i + (lane >> 3);
+    const int mg = m_blk * BM + m;
+    const int nv = (mg < g.Mr) ? kvalid : 0;
+    v[i] = fetch_seg16(g.a + static_cast<int64_t>(mg) * g.lda + k0, gl, 8, nv, g.a_lo, g.a_hi);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = lw * 32 + 4 * i + (lane >> 3);
+    uint8_t* p = dst + m * 128 + ((gl ^ (m & 7)) << 4);
+    *reinterpret_cast<uint4*>(p) = v[i];
+  }
+}
+
+// Manual load of Bop's [64 × 256] MN-major tile: each loader warp fills 16
+// rows (k), one 512-byte row segment (32 lanes × 16 B) per instruction.
+__device__ __forceinline__ void load_b_manual(uint8_t* dst, const GemmArgs& g, int n_blk, int kb,
+                                              int lw, int lane) {
+  const int n0 = n_blk * BN;
+  const int nvalid = min(BN, g.Nc - n0);
+  constexpr int U = 8;
+#pragma unroll
+  for (int i0 = 0; i0 < 16; i0 += U) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = lw + LOADER_WARPS * (i0 + u);
+      const int kg = kb * BK + k;
+      const int nv = (kg < g.Kc) ? nvalid : 0;
+      v[u] = fetch_seg16(g.b + static_cast<int64_t>(kg) * g.ldb + n0, lane, 32, nv, g.b_lo, g.b_hi);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = lw + LOADER_WARPS * (i0 + u);
+      uint8_t* p = dst + (lane >> 3) * B_ATOM + k * 128 + (((lane & 7) ^ (k & 7)) << 4);
+      *reinterpret_cast<uint4*>(p) = v[u];
+    }
+  }
+}
+
+__device__ __forceinline__ void store_chunk(const GemmArgs& g, int row, int col0,
+                                            const uint32_t (&v)[32], bool vec_ok) {
+  if (row >= g.Mr) return;
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+  if (g.bias) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = col0 + i;
+      if (c < g.Nc) f[i] += __bfloat162float(g.bias[c]);
+    }
+  }
+  __nv_bfloat16* dst = g.c + static_cast<int64_t>(row) * g.ldc + col0;
+  if (vec_ok && col0 + 32 <= g.Nc) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16x2(f[8 * q + 0], f[8 * q + 1]);
+      w.y = pack_bf16x2(f[8 * q + 2], f[8 * q + 3]);
+      w.z = pack_bf16x2(f[8 * q + 4], f[8 * q + 5]);
+      w.w = pack_bf16x2(f[8 * q + 6], f[8 * q + 7]);
+      *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col0 + i < g.Nc) dst[i] = __float2bfloat16_rn(f[i]);
+  }
+}
+
+template <bool A_TMA, bool B_TMA>
+struct GemmCfg {
+  static constexpr bool kAnyManual = !A_TMA || !B_TMA;
+  static constexpr bool kAnyTma = A_TMA || B_TMA;
+  static constexpr int kWarps = 6 + (kAnyManual ? LOADER_WARPS : 0);
+  static constexpr int kThreads = kWarps * 32;
+};
+
+template <bool A_TMA, bool B_TMA>
+__global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                     const __grid_constant__ CUtensorMap map_b, const GemmArgs g) {
+  using Cfg = GemmCfg<A_TMA, B_TMA>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  Smem sm{smem_raw + (((raw + 1023u) & ~1023u) - raw)};
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm.base + STAGES * STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* fin = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], (Cfg::kAnyTma ? 1u : 0u) + (Cfg::kAnyManual ? LOADER_WARPS : 0u));
+      mbar_init(&empty[s], 1u);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1u);
+      mbar_init(&tempty[i], EPI_WARPS);
+    }
+    mbar_init(fin, 1u);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == TMA_WARP && lane == 0) {
+    if (A_TMA) tma_prefetch_desc(&map_a);
+    if (B_TMA) tma_prefetch_desc(&map_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int num_tiles = g.tiles_m * g.tiles_n;
+  const int num_kb = (g.Kc + BK - 1) / BK;
+  // Producer bookkeeping for a clean exit after a timeout.
+  int issued_phase[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
+  bool ok = true;
+
+  if (warp == TMA_WARP) {
+    if (Cfg::kAnyTma && lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], (A_TMA ? A_STAGE : 0) + (B_TMA ? B_STAGE : 0));
+          if (A_TMA) tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
+          if (B_TMA) {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
+          }
+          issued_phase[s] = static_cast<int>(ph);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (Cfg::kAnyManual && warp >= LOADER_WARP0) {
+    const int lw = warp - LOADER_WARP0;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereLoader)) {
+          ok = false;
+          break;
+        }
+        if (!A_TMA) load_a_manual(sm.a(s), g, m_blk, kb, lw, lane);
+        if (!B_TMA) load_b_manual(sm.b(s), g, n_blk, kb, lw, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    const uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
+    int s = 0;
+    uint32_t ph = 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
+      if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait, kWhereMmaAcc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full[s], ph, g.wait, kWhereMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const int krem = g.Kc - kb * BK;
+          const int nk = krem >= BK ? BK / 16 : (krem + 15) / 16;
+          const uint32_t a0 = smem_u32(sm.a(s));
+          const uint32_t b0 = smem_u32(sm.b(s));
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, B_ATOM, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        __syncwarp();
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&tfull[acc]);
+      __syncwarp();
+    }
+  } else if (warp < EPI_WARPS) {
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(g.c) & 15u) == 0) && ((g.ldc & 7) == 0);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
+      const int acc = it & 1;
+      const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
+      if (!mbar_wait(&tfull[acc], aph, g.wait, kWhereEpilogue)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = m_blk * BM + warp * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = n_blk * BN + c * 32;
+        if (col0 >= g.Nc) break;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
+        tmem_ld_wait();
+        store_chunk(g, row, col0, v, vec_ok);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  // Teardown.  Every wait above is bounded, so every thread gets here.
+  if (warp == MMA_WARP && lane == 0) {
+    // All MMAs this thread issued are complete once fin flips.
+    umma_commit(fin);
+    mbar_wait_drain(fin, 0u, 2000000000ull);
+  }
+  if (warp == TMA_WARP && lane == 0 && !ok) {
+    // After a timeout: let any TMA load still in flight land before exit.
+    for (int s = 0; s < STAGES; ++s)
+      if (issued_phase[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_phase[s]), 1000000ull);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+__global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+                                 const __nv_bfloat16* bias) {
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, n = i % N;
+    Y[m * ldy + n] = bias ? bias[n] : __float2bfloat16_rn(0.f);
+  }
+}
+
+template <bool A_TMA, bool B_TMA>
+cudaError_t launch_impl(const GemmArgs& g, const GemmMaps& maps, int num_sms,
+                        cudaStream_t stream) {
+  using Cfg = GemmCfg<A_TMA, B_TMA>;
+  auto kern = umma_gemm_kernel<A_TMA, B_TMA>;
+  const size_t smem = gemm_smem_bytes();
+  cudaError_t e = ensure_max_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int tiles = g.tiles_m * g.tiles_n;
+  const int grid = std::max(1, std::min(tiles, num_sms));
+  kern<<<grid, Cfg::kThreads, smem, stream>>>(maps.a, maps.b, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes() {
+  return 1024 + static_cast<size_t>(STAGES) * STAGE + (2 * STAGES + 5) * sizeof(uint64_t) + 16;
+}
+
+cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,
+                        cudaStream_t stream) {
+  if (maps.a_tma && maps.b_tma) return launch_impl<true, true>(g, maps, num_sms, stream);
+  if (maps.a_tma) return launch_impl<true, false>(g, maps, num_sms, stream);
+  if (maps.b_tma) return launch_impl<false, true>(g, maps, num_sms, stream);
+  return launch_impl<false, false>(g, maps, num_sms, stream);
+}
+
+cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+                             const __nv_bfloat16* bias, cudaStream_t stream) {
+  const int64_t total = M * N;
+  const int threads = 256;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 4096));
+  fill_bias_kernel<<<std::max(blocks, 1), threads, 0, stream>>>(Y, ldy, M, N, bias);
+  return cudaGetLastError();
+}
+
+}  // namespace lr

@@ -1,0 +1,97 @@
+"""The C-ABI library loads and exports every declared symbol (no GPU needed),
+and argument errors come back before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rank_linear_layers_b200 as lr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(lr_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from rank_linear_layers_b200 import build
+    if build.needs_build():
+        build.build()
+    return lr.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared()
+    assert declared, "no declarations found"
+    for name in declared:
+        assert hasattr(L, name), f"missing export {name}"
+    assert declared == set(lr.EXPORTS)
+
+
+def test_status_strings(L):
+    assert lr.status_string(lr.LR_OK) == "LR_OK"
+    assert lr.status_string(lr.LR_ERR_TIMEOUT) == "LR_ERR_TIMEOUT"
+    assert lr.status_string(99) == "LR_ERR_UNKNOWN"
+
+
+def test_invalid_arguments_rejected_before_cuda(L):
+    p = ctypes.c_void_p(0x1000)
+    # Negative sizes.
+    assert L.lr_linear(p, p, p, None, p, -1, 4, 4, 4, None) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_linear(p, p, p, None, p, 4, 4, -3, 4, None) == lr.LR_ERR_INVALID_ARG
+    # Null inputs with a nonempty problem.
+    assert L.lr_linear(None, p, p, None, p, 4, 4, 4, 4, None) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_linear(p, p, p, None, None, 4, 4, 4, 4, None) == lr.LR_ERR_INVALID_ARG
+    # Odd (not 2-byte aligned) pointer.
+    assert L.lr_linear(ctypes.c_void_p(0x1001), p, ctypes.c_void_p(0x9000), None,
+                       ctypes.c_void_p(0x20000), 4, 4, 4, 4, None) == lr.LR_ERR_INVALID_ARG
+    # Y overlapping X.
+    assert L.lr_linear(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x8000), ctypes.c_void_p(0x9000),
+                       None, ctypes.c_void_p(0x1004), 4, 4, 4, 4, None) == lr.LR_ERR_INVALID_ARG
+    # Sizes past int32 are unsupported.
+    assert L.lr_linear(p, p, p, None, p, 1 << 31, 4, 4, 4, None) == lr.LR_ERR_UNSUPPORTED
+    # Empty problems are a no-op that needs no device.
+    assert L.lr_linear(None, None, None, None, None, 0, 4, 4, 4, None) == lr.LR_OK
+    assert L.lr_linear(None, None, None, None, None, 4, 4, 4, 0, None) == lr.LR_OK
+    # Group: bad count, and two projections writing the same elements.
+    assert L.lr_linear_group(None, -1, 4, None) == lr.LR_ERR_INVALID_ARG
+    arr = (lr.LrProj * 2)()
+    for i in range(2):
+        arr[i] = lr.LrProj(0x100000, 8, 0x200000, 0x300000, None, 0x400000, 16, 4, 16)
+    assert L.lr_linear_group(arr, 2, 4, None) == lr.LR_ERR_INVALID_ARG
+
+
+def test_packed_halves_are_accepted_by_validation(L):
+    # gate and up write the two halves of one [M, 2N] buffer: disjoint, valid.
+    # Validation passes; without a device the call then fails on CUDA, not on
+    # the arguments.
+    arr = (lr.LrProj * 2)()
+    N = 12203
+    arr[0] = lr.LrProj(0x100000, 8, 0x200000, 0x300000, None, 0x4000000, 2 * N, 4, N)
+    arr[1] = lr.LrProj(0x100000, 8, 0x210000, 0x310000, None, 0x4000000 + 2 * N, 2 * N, 4, N)
+    assert L.lr_linear_group(arr, 2, 3, None) != lr.LR_ERR_INVALID_ARG
+    # Shift the second half left by one element: now they share a column.
+    arr[1] = lr.LrProj(0x100000, 8, 0x210000, 0x310000, None, 0x4000000 + 2 * N - 2, 2 * N, 4, N)
+    assert L.lr_linear_group(arr, 2, 3, None) == lr.LR_ERR_INVALID_ARG
+
+
+def test_controls(L):
+    assert L.lr_set_path(7) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_set_path(0) == lr.LR_OK
+    assert L.lr_set_wait_limit_ns(-1) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_set_wait_limit_ns(0) == lr.LR_OK
+    assert L.lr_kernel_launch_count() >= 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError):
+        lr.lib(str(tmp_path / "missing.so"))

@@ -1,0 +1,166 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar (bf16 inputs, fp32 accumulation): max|err| <= 2e-2·RMS(Y_ref) and
+relative Frobenius error <= 5e-3, on every output (tests/helpers.py).
+Small cases compare every element; full-size workloads compare sampled rows,
+which the oracle computes one by one (each output row depends only on its X
+row).
+"""
+import numpy as np
+import pytest
+
+import lrgen
+import oracle
+from helpers import compare, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lr():
+    import torch
+    import rank_linear_layers_b200 as lr
+    lr.set_path(lr.PATH_AUTO)
+    yield lr
+    lr.set_path(lr.PATH_AUTO)
+    torch.cuda.synchronize()
+
+
+def run_gpu(lr, p, path=0, bias=None):
+    import torch
+    lr.set_path(path)
+    try:
+        X, A, B = to_dev(p["X"]), to_dev(p["A"]), to_dev(p["B"])
+        b = to_dev(p["bias"] if bias is None else bias)
+        Y = lr.lr_linear(X, A, B, b)
+        torch.cuda.synchronize()
+        assert lr.last_device_status() == lr.LR_OK
+        return to_f64(Y)
+    finally:
+        lr.set_path(0)
+
+
+def ref(p, rows=None):
+    return oracle.lr_linear(p["X"], p["A"], p["B"], p["bias"], rows=rows)
+
+
+# ---------------------------------------------------------------- decode
+def test_single_layer_m16_k256_r107(lr):
+    # X [16,256] ~N(0,1), A [256,107], B [107,256] ~N(0,1/fan_in), no bias, seed 0.
+    p = lrgen.lowrank_problem(16, 256, 107, 256, seed=0)
+    Yr = ref(p)
+    compare(run_gpu(lr, p), Yr, "c1 auto")
+    compare(run_gpu(lr, p, lr.PATH_DECODE), Yr, "c1 decode")
+    compare(run_gpu(lr, p, lr.PATH_PREFILL), Yr, "c1 prefill")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 16])
+@pytest.mark.parametrize("r", [1, 7, 8, 9, 63, 65, 107, 255, 257, 300])
+def test_decode_ragged(lr, M, r):
+    K, N = 333, 517
+    p = lrgen.lowrank_problem(M, K, r, N, seed=1000 + r, bias=(r % 2 == 1))
+    compare(run_gpu(lr, p, lr.PATH_DECODE), ref(p), f"decode M={M} r={r}")
+
+
+@pytest.mark.parametrize("K,N", [(8, 8), (1, 1000), (4096, 40), (130, 2049)])
+def test_decode_shapes(lr, K, N):
+    p = lrgen.lowrank_problem(4, K, 37, N, seed=7, bias=True)
+    compare(run_gpu(lr, p, lr.PATH_DECODE), ref(p), f"decode K={K} N={N}")
+    p = lrgen.lowrank_problem(16, K, 37, N, seed=8, bias=True)
+    compare(run_gpu(lr, p, lr.PATH_DECODE), ref(p), f"decode16 K={K} N={N}")
+
+
+# ---------------------------------------------------------------- prefill
+@pytest.mark.parametrize("M,K,r,N", [
+    (128, 64, 64, 256),       # one tile each way, all aligned
+    (128, 128, 256, 256),
+    (200, 256, 107, 300),     # odd r (A rows 2-byte aligned), ragged M and N
+    (300, 333, 257, 517),     # odd K too (X rows misaligned)
+    (17, 64, 1, 8),           # smallest prefill M, rank 1
+    (129, 1000, 511, 1000),
+    (256, 512, 1741 // 4, 700),
+    (384, 4096, 1741, 256),   # full-depth K, c2's rank
+])
+def test_prefill_ragged(lr, M, K, r, N):
+    p = lrgen.lowrank_problem(M, K, r, N, seed=M + K + r + N, bias=True)
+    compare(run_gpu(lr, p, lr.PATH_PREFILL), ref(p), f"prefill {M}x{K}x{r}x{N}")
+
+
+def test_decode_and_prefill_agree_at_m16(lr):
+    p = lrgen.lowrank_problem(16, 512, 300, 640, seed=3, bias=True)
+    Yd = run_gpu(lr, p, lr.PATH_DECODE)
+    Yp = run_gpu(lr, p, lr.PATH_PREFILL)
+    Yr = ref(p)
+    compare(Yd, Yr, "decode")
+    compare(Yp, Yr, "prefill")
+    compare(Yd, Yp, "decode vs prefill")
+
+
+# ---------------------------------------------------------------- edges
+def test_empty_and_degenerate(lr):
+    import torch
+    # r = 0 and K = 0: Y = bias.
+    for (M, K, r, N) in [(5, 8, 0, 9), (40, 0, 3, 9), (3, 0, 0, 4)]:
+        p = lrgen.lowrank_problem(M, K, r, N, seed=1, bias=True)
+        X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+        A = torch.zeros((K, r), dtype=torch.bfloat16, device="cuda")
+        B = torch.zeros((r, N), dtype=torch.bfloat16, device="cuda")
+        b = to_dev(p["bias"])
+        Y = lr.lr_linear(X, A, B, b)
+        assert np.array_equal(to_f64(Y), np.broadcast_to(lrgen.bf16_to_f64(p["bias"]), (M, N)))
+    # M = 0 or N = 0: nothing to do.
+    X = torch.zeros((0, 8), dtype=torch.bfloat16, device="cuda")
+    Y = lr.lr_linear(X, torch.zeros((8, 3), dtype=torch.bfloat16, device="cuda"),
+                     torch.zeros((3, 5), dtype=torch.bfloat16, device="cuda"))
+    assert Y.shape == (0, 5)
+
+
+def test_unaligned_base_pointers(lr):
+    """Views that start 2 bytes into a buffer: no operand is 16-byte aligned."""
+    import torch
+    for (M, K, r, N, path) in [(200, 136, 64, 264, 2), (8, 136, 64, 264, 1)]:
+        p = lrgen.lowrank_problem(M, K, r, N, seed=21, bias=True)
+        def off(bits):
+            t = to_dev(bits).reshape(-1)
+            buf = torch.empty(t.numel() + 1, dtype=torch.bfloat16, device="cuda")
+            buf[1:] = t
+            return buf[1:].view(bits.shape)
+        X, A, B, b = off(p["X"]), off(p["A"]), off(p["B"]), off(p["bias"])
+        ybuf = torch.empty(M * N + 1, dtype=torch.bfloat16, device="cuda")
+        Y = ybuf[1:].view(M, N)
+        assert X.data_ptr() % 16 != 0 and Y.data_ptr() % 16 != 0
+        lr.set_path(path)
+        try:
+            lr.lr_linear(X, A, B, b, Y=Y)
+        finally:
+            lr.set_path(0)
+        torch.cuda.synchronize()
+        compare(to_f64(Y), ref(p), f"unaligned path={path}")
+
+
+def test_repeated_calls_reuse_workspace(lr):
+    """The decode workspace must be zero again after each call (self-cleaning)."""
+    p = lrgen.lowrank_problem(4, 1024, 300, 2000, seed=5)
+    q = lrgen.lowrank_problem(16, 700, 1000, 129, seed=6, bias=True)
+    Yp, Yq = ref(p), ref(q)
+    for _ in range(3):
+        compare(run_gpu(lr, p, lr.PATH_DECODE), Yp, "p")
+        compare(run_gpu(lr, q, lr.PATH_DECODE), Yq, "q")
+
+
+# ---------------------------------------------------------------- full size
+def test_prefill_q_proj_full_size_sampled_rows(lr):
+    # M=2048, K=N=4096, r=1741; A = U·Σ, B = Vᵀ with σ_i = i^-0.5.
+    p = lrgen.svd_problem(M=2048, K=4096, N=4096, r=1741, seed=0)
+    Y = run_gpu(lr, p)
+    rows = np.random.default_rng(0).choice(2048, 96, replace=False)
+    rows = np.concatenate([rows, [0, 127, 128, 2047]])
+    compare(Y[rows], ref(p, rows=rows), "q_proj sampled rows")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("proj", ["gate_up", "down"])
+def test_decode_mlp_full_size(lr, M, proj):
+    K, N = (4096, 14336) if proj == "gate_up" else (14336, 4096)
+    p = lrgen.lowrank_problem(M, K, 2867, N, seed=0)
+    compare(run_gpu(lr, p), ref(p), f"decode {proj} M={M}")
