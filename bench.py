@@ -1,0 +1,438 @@
+"""Benchmark of the low-rank linear layer Y = (X·A)·B on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step = one lr_linear call over one batch): the prefill q_proj
+shape of Llama-3-8B, X [2048, 4096] ~ N(0,1), A = U·Σ [4096, 1741],
+B = Vᵀ [1741, 4096], U and V Haar orthogonal, σ_i = i^-0.5 (bf16 inputs,
+fp32 accumulation).  Rank 1741 is not a multiple of 8: keeping 15% fewer
+parameters than the 4096×4096 layer, as in the GAC paper's ASVD setting.
+
+Prints one JSON line (rank 0).  `value` is whole-job TFLOP/s (2·M·r·(K+N)
+FLOPs per step per rank, summed over ranks, over the max-over-ranks device
+time).  Inputs rotate over enough copies to exceed twice the L2 size, so no
+step reads its operands from L2.  Also reported: the roofline fraction of the
+prefill kernels, the end-to-end rate through the host-buffer C ABI call, the
+decode (M = 1, 4, 16) bandwidth of the Llama-3-8B MLP shapes, the fp64 CPU
+oracle timed on a bounded sample (the CPU baseline), SM clocks sampled during
+the timed region and the number of library kernels launched.
+
+With --gpus N > 1 (torchrun), every rank runs its own batch with the same
+factors (rows of X are independent): weak scaling, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import lrgen  # noqa: E402
+from rank_linear_layers_b200 import accounting as acc  # noqa: E402
+
+M, K, R, N = 2048, 4096, 1741, 4096
+WORKLOAD = "prefill q_proj: X[2048,4096] · A[4096,1741] (U·Σ, σ_i=i^-0.5) · B[1741,4096] (Vᵀ), bf16"
+CACHE = os.environ.get("LR_BENCH_CACHE", "/tmp/lr_bench_inputs")
+DECODE_SHAPES = [("gate_up", 4096, 2867, 14336), ("down", 14336, 2867, 4096)]
+
+
+def fallback_peaks():
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except Exception:
+        return fallback_peaks()
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_linear_layers_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        vals = {}
+        for line in open(path):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+        if vals.get("kernel_source_hash") != kernel_source_hash():
+            return None
+        return float(vals["dram_bytes_per_step"])
+    except Exception:
+        return None
+
+
+def prefill_inputs():
+    """The prefill problem (cached on disk: the QR of two 4096² matrices takes a while)."""
+    os.makedirs(CACHE, exist_ok=True)
+    f = os.path.join(CACHE, f"q_proj_{M}_{K}_{R}_{N}_seed0.npz")
+    if os.path.exists(f):
+        z = np.load(f)
+        return {"X": z["X"], "A": z["A"], "B": z["B"], "bias": None}
+    p = lrgen.svd_problem(M=M, K=K, N=N, r=R, seed=0)
+    try:
+        np.savez(f + ".tmp.npz", X=p["X"], A=p["A"], B=p["B"])
+        os.replace(f + ".tmp.npz", f)
+    except OSError:
+        pass
+    return p
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- timing
+def time_steps(fn, steps, warmup, flush=None):
+    """Device time of `steps` calls (CUDA events on the launching stream)."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        fn(warmup + i)
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e-3
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _reduce(x, world, op):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def max_over_ranks(x, world):
+    """Timing across ranks: the slowest rank's device time."""
+    import torch.distributed as dist
+    return x if world == 1 else _reduce(x, world, dist.ReduceOp.MAX)
+
+
+def sum_over_ranks(x, world):
+    """Work across ranks: every rank's units count."""
+    import torch.distributed as dist
+    return x if world == 1 else _reduce(x, world, dist.ReduceOp.SUM)
+
+
+def aggregate(flops_per_rank, seconds_per_rank, world):
+    """Whole-job TFLOP/s: units of all ranks over the max-over-ranks time."""
+    t = max_over_ranks(seconds_per_rank, world)
+    return sum_over_ranks(flops_per_rank, world) / t / 1e12, t
+
+
+# ---------------------------------------------------------------- CPU baseline
+def cpu_baseline(p, budget_s=12.0):
+    """The fp64 oracle on a bounded row sample of the same workload."""
+    import oracle
+    threads = oracle.default_threads()
+    rows_per_chunk = 32
+    done = 0
+    t0 = time.perf_counter()
+    rng = np.random.default_rng(1)
+    while time.perf_counter() - t0 < budget_s and done < 4 * M:
+        rows = rng.choice(M, rows_per_chunk, replace=False)
+        oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rows, threads=threads)
+        done += rows_per_chunk
+    dt = time.perf_counter() - t0
+    fl = acc.flops(done, K, R, N)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} rows of X (of {M}) through the fp64 oracle, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    p = prefill_inputs()
+    # Each step is one bounded sample; time K of them after W warm-ups.
+    import oracle
+    threads = oracle.default_threads()
+    rows_per_step = 64
+    rng = np.random.default_rng(2)
+    for _ in range(args.warmup):
+        oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rng.choice(M, rows_per_step, replace=False),
+                         threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rng.choice(M, rows_per_step, replace=False),
+                         threads=threads)
+    dt = time.perf_counter() - t0
+    value = acc.flops(rows_per_step * args.steps, K, R, N) / dt / 1e12
+    cb = {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+          "sample": f"{rows_per_step} rows of X per step (of {M}), fp64 oracle"}
+    line = {
+        "impl": "reference", "metric": metric_name(), "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / max(1, args.steps) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(), "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def metric_name():
+    return "low-rank linear TFLOP/s (prefill) and GB/s (decode) as % of B200 roofline"
+
+
+def config_dict():
+    return {"workload": WORKLOAD, "M": M, "K": K, "r": R, "N": N, "r_mod_8": R % 8,
+            "factors": "A=U·Σ, B=Vᵀ, Haar U,V, sigma_i=i^-0.5", "bias": False,
+            "l2": "inputs rotate over copies totalling > 2x L2 between steps",
+            "parallelism": "data-parallel rows of X, factors replicated (weak scaling)"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import rank_linear_layers_b200 as lr
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    p = prefill_inputs()
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X0, A0, B0 = to_dev(p["X"]), to_dev(p["A"]), to_dev(p["B"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    step_bytes = (X0.numel() + A0.numel() + B0.numel()) * 2
+    copies = max(2, math.ceil(2 * l2 / step_bytes) + 1)
+    Xs = [X0] + [X0.clone() for _ in range(copies - 1)]
+    As = [A0] + [A0.clone() for _ in range(copies - 1)]
+    Bs = [B0] + [B0.clone() for _ in range(copies - 1)]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        j = i % copies
+        lr.lr_linear(Xs[j], As[j], Bs[j], None, Y=Y)
+
+    # Correctness gate on the timed configuration: sampled rows vs the oracle.
+    step(0)
+    torch.cuda.synchronize()
+    if lr.last_device_status() != lr.LR_OK:
+        raise RuntimeError("device status not OK")
+    parity = None
+    if rank == 0:
+        import oracle
+        rows = np.random.default_rng(0).choice(M, 16, replace=False)
+        Yr = oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rows)
+        Yg = lrgen.bf16_to_f64(Y[torch.as_tensor(rows, device=dev)].cpu().view(torch.int16).numpy().view(np.uint16))
+        rms = float(np.sqrt(np.mean(Yr ** 2)))
+        parity = {"rows": 16, "max_err_over_rms": float(np.abs(Yg - Yr).max() / rms),
+                  "rel_fro": float(np.linalg.norm(Yg - Yr) / np.linalg.norm(Yr))}
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches0 = lr.kernel_launch_count()
+    t = time_steps(step, args.steps, 0)
+    launches_timed = lr.kernel_launch_count() - launches0
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    fl_step = acc.flops(M, K, R, N)
+    value, t_max = aggregate(fl_step * args.steps, t, world)
+    ms = t_max / args.steps * 1e3
+
+    # Roofline of the prefill kernels: two launches of the tcgen05 GEMM per
+    # step (T = X·A, then Y = T·B), each doing half of the step's FLOPs.
+    peak = peaks.get("bf16_tflops") or fallback_peaks()["bf16_tflops"]
+    achieved = fl_step / (t / args.steps) / 1e12
+    traffic = recorded_traffic("umma_gemm_prefill_q_proj.txt")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_kind": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
+                "kernel": "umma_gemm_kernel x2 per step (GEMM1 T=X·A, GEMM2 Y=T·B)",
+                "algorithmic_bytes_per_step": acc.algorithmic_bytes(M, K, R, N),
+                "flops_per_step": fl_step}
+
+    # End to end through the host-buffer C ABI call (pinned host memory).
+    e2e = None
+    try:
+        Xh = torch.from_numpy(p["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        Ah = torch.from_numpy(p["A"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        Bh = torch.from_numpy(p["B"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            lr.lr_linear_host(Xh, Ah, Bh, None, Y=Yh)
+        barrier(world)
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            lr.lr_linear_host(Xh, Ah, Bh, None, Y=Yh)
+        te = max_over_ranks((time.perf_counter() - t0) / e2e_steps, world)
+        e2e = {"value": sum_over_ranks(fl_step, world) / te / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int((Xh.numel() + Ah.numel() + Bh.numel()) * 2),
+               "d2h_bytes_per_step": int(Yh.numel() * 2), "ms_per_step": te * 1e3,
+               "steps": e2e_steps, "note": "lr_linear_host: X, A, B copied in and Y out every step"}
+    except Exception as ex:  # pragma: no cover - reported, not hidden
+        e2e = {"value": None, "unit": "TFLOP/s", "error": str(ex)[:200]}
+
+    # Decode (M = 1, 4, 16) on the MLP shapes: bandwidth and % of HBM peak.
+    decode = {}
+    if not args.no_decode:
+        for name, dk, dr, dn in DECODE_SHAPES:
+            for dm in (1, 4, 16):
+                q = lrgen.lowrank_problem(dm, dk, dr, dn, seed=0)
+                Xd, Ad, Bd = to_dev(q["X"]), to_dev(q["A"]), to_dev(q["B"])
+                cps = max(2, math.ceil(2 * l2 / ((Ad.numel() + Bd.numel()) * 2)) + 1)
+                Ads = [Ad] + [Ad.clone() for _ in range(cps - 1)]
+                Bds = [Bd] + [Bd.clone() for _ in range(cps - 1)]
+                Yd = torch.empty((dm, dn), dtype=torch.bfloat16, device=dev)
+
+                def dstep(i, Xd=Xd, Ads=Ads, Bds=Bds, Yd=Yd, cps=cps):
+                    lr.lr_linear(Xd, Ads[i % cps], Bds[i % cps], None, Y=Yd)
+                td = time_steps(dstep, 50, 5) / 50
+                by = acc.algorithmic_bytes(dm, dk, dr, dn)
+                decode[f"{name}_M{dm}"] = {
+                    "us": td * 1e6, "GB/s": by / td / 1e9,
+                    "frac_hbm": by / td / 1e9 / peaks["hbm_gbs"],
+                    "dense_equiv_us_at_peak": acc.dense_bytes(dm, dk, dn) / (peaks["hbm_gbs"] * 1e9) * 1e6}
+                del Ads, Bds
+
+    cb = cpu_baseline(p) if (rank == 0 and world == 1) else None
+    if rank == 0:
+        line = {
+            "metric": metric_name(), "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_dict(), "roofline": roofline,
+            "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches_timed),
+            "clocks": clk, "parity": parity, "decode": decode,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

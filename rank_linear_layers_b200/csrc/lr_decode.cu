@@ -100,12 +100,14 @@ __device__ __forceinline__ void reduce_and_finalise(const SkinnyArgs& a, float* 
 
 // ---------------------------------------------------------------- FMA path
 // One warp reads one 256-column row segment (32 lanes × 8 columns); the 8
-// warps take rows round robin.
+// warps take rows round robin, each with U rows in flight.
+constexpr int kFmaU = 8;
+
 template <int MT>
-__global__ void __launch_bounds__(kWarps * 32) skinny_fma_kernel(SkinnyArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 2) skinny_fma_kernel(SkinnyArgs a) {
   constexpr int CW = 8;
   constexpr int COLS = 32 * CW;
-  constexpr int U = 4;  // rows in flight per warp
+  constexpr int U = kFmaU;
   extern __shared__ __align__(16) float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * COLS;
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(kWarps * 32) skinny_fma_kernel(SkinnyArgs a) {
   stage_v_kmajor<MT>(sv, a, k0, kc, a.k_chunk);
   __syncthreads();
 
-  // acc2[m/2][c] holds (token m, token m+1) for column c (FFMA2 pairs over m).
+  // acc[m/2][c] holds (token m, token m+1) for column c (FFMA2 pairs over m).
   constexpr int MP = (MT + 1) / 2;
   float2 acc[MP][CW];
 #pragma unroll
@@ -127,35 +129,40 @@ __global__ void __launch_bounds__(kWarps * 32) skinny_fma_kernel(SkinnyArgs a) {
 
   const __nv_bfloat16* wbase = a.W + n0;
   for (int kk = warp; kk < kc; kk += kWarps * U) {
-    uint4 w[U];
+    uint4 cur[U], ext[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int k = kk + u * kWarps;
       const int nv = (k < kc) ? nvalid : 0;
-      w[u] = fetch_seg16(wbase + (k0 + k) * a.ldw, lane, 32, nv, a.w_lo, a.w_hi);
+      seg16_issue(wbase + (k0 + k) * a.ldw, lane, 32, nv, a.w_lo, a.w_hi, cur[u], ext[u]);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int k = kk + u * kWarps;
       if (k >= kc) break;
+      const __nv_bfloat16* rowp = wbase + (k0 + k) * a.ldw;
+      const uint4 w = seg16_finish(cur[u], ext[u], seg_shift(rowp), lane, 32, nvalid);
       const float* vrow = sv + k * MT;
       float wf[CW];
-      const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         wf[2 * i] = bf16lo_to_f32(ww[i]);
         wf[2 * i + 1] = bf16hi_to_f32(ww[i]);
       }
+      if (MT == 1) {
+        // One token: plain FMA, acc[0][c].x only.
+        const float v = vrow[0];
 #pragma unroll
-      for (int p = 0; p < MP; ++p) {
-        float2 vv;
-        if (MT == 1) {
-          vv = make_float2(vrow[0], 0.f);
-        } else {
-          vv = *reinterpret_cast<const float2*>(vrow + 2 * p);
+        for (int c = 0; c < CW; ++c) acc[0][c].x = fmaf(v, wf[c], acc[0][c].x);
+      } else {
+#pragma unroll
+        for (int p = 0; p < MP; ++p) {
+          const float2 vv = *reinterpret_cast<const float2*>(vrow + 2 * p);
+#pragma unroll
+          for (int c = 0; c < CW; ++c)
+            acc[p][c] = __ffma2_rn(vv, make_float2(wf[c], wf[c]), acc[p][c]);
         }
-#pragma unroll
-        for (int c = 0; c < CW; ++c) acc[p][c] = __ffma2_rn(vv, make_float2(wf[c], wf[c]), acc[p][c]);
       }
     }
   }
@@ -181,12 +188,15 @@ __global__ void __launch_bounds__(kWarps * 32) skinny_fma_kernel(SkinnyArgs a) {
 }
 
 // ---------------------------------------------------------------- MMA path
-// One warp owns 16-row steps of the CTA's row range; a step reads 16 rows ×
-// 128 columns (two rows per load instruction, 16 lanes per row), writes them
-// to the warp's shared buffer, and runs 16 mma.m16n8k16 (32 in phase 2).
-constexpr int kMmaCols = 128;
+// The CTA owns 64 columns.  A warp step covers 16 rows of W: four load
+// instructions of four rows each (8 lanes × 16 B per row), realigned, stored
+// to the warp's shared buffer, then read back with ldmatrix.trans as the B
+// fragments of 8 mma.m16n8k16 (16 in phase 2).  Two steps are in flight per
+// warp (the next step's loads are issued before this step's MMAs).
+constexpr int kMmaCols = 64;
 constexpr int kMmaRowBytes = kMmaCols * 2 + 16;  // padded: conflict-free ldmatrix
 constexpr int kMmaBufBytes = 16 * kMmaRowBytes;
+constexpr int kMmaStep = 16 * kWarps;            // rows between a warp's steps
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
@@ -204,8 +214,78 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                : "r"(addr));
 }
 
+struct MmaCtx {
+  const __nv_bfloat16* wbase;  // W + n0
+  int64_t k0, ldw;
+  int kc, nvalid;
+  uintptr_t lo, hi;
+  int rg, g8;  // row within a load instruction (0..3), lane within the row (0..7)
+};
+
+__device__ __forceinline__ void mma_issue(const MmaCtx& c, int ks, uint4 (&cur)[4],
+                                          uint4 (&ext)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = ks + 4 * i + c.rg;
+    const int nv = (k < c.kc) ? c.nvalid : 0;
+    seg16_issue(c.wbase + (c.k0 + k) * c.ldw, c.g8, 8, nv, c.lo, c.hi, cur[i], ext[i]);
+  }
+}
+
 template <bool V_F32>
-__global__ void __launch_bounds__(kWarps * 32) skinny_mma_kernel(SkinnyArgs a) {
+__device__ __forceinline__ void mma_step(const MmaCtx& c, int ks, const uint4 (&cur)[4],
+                                         const uint4 (&ext)[4], uint8_t* tbuf, const float* sv,
+                                         float (&d)[8][4], int lane) {
+  constexpr int MT = 16;
+  // 1. Realign the 16 rows into the warp buffer.
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 4 * i + c.rg;
+    const int k = ks + row;
+    const int nv = (k < c.kc) ? c.nvalid : 0;
+    const uint4 w = seg16_finish(cur[i], ext[i], seg_shift(c.wbase + (c.k0 + k) * c.ldw), c.g8, 8, nv);
+    *reinterpret_cast<uint4*>(tbuf + row * kMmaRowBytes + c.g8 * 16) = w;
+  }
+  __syncwarp();
+  // 2. A fragment (tokens × 16 rows of W) from the staged V.
+  const int g = lane >> 2, tq = lane & 3;
+  uint32_t ahi[4], alo[4];
+  {
+    const float* v0 = sv + (ks + 2 * tq) * MT;
+    const float* v1 = v0 + MT;
+    const float* v8 = v0 + 8 * MT;
+    const float* v9 = v8 + MT;
+    const float f[8] = {v0[g], v1[g], v0[g + 8], v1[g + 8], v8[g], v9[g], v8[g + 8], v9[g + 8]};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t h = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+      ahi[i] = h;
+      if (V_F32) {
+        alo[i] = pack_bf16x2(f[2 * i] - bf16lo_to_f32(h), f[2 * i + 1] - bf16hi_to_f32(h));
+      }
+    }
+  }
+  // 3. B fragments via ldmatrix.trans; matrix j = lane/8 covers rows
+  // (j&1)*8 .. +7 and columns (j>>1)*8 .. +7 of a 16×16 block.
+  const uint32_t tb = smem_u32(tbuf);
+  const int lm_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int lm_col = (lane >> 4) * 8;
+#pragma unroll
+  for (int nb = 0; nb < kMmaCols / 16; ++nb) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_trans(tb + lm_row * kMmaRowBytes + (nb * 16 + lm_col) * 2, b0, b1, b2, b3);
+    mma_bf16_16816(d[2 * nb], ahi, b0, b1);
+    mma_bf16_16816(d[2 * nb + 1], ahi, b2, b3);
+    if (V_F32) {
+      mma_bf16_16816(d[2 * nb], alo, b0, b1);
+      mma_bf16_16816(d[2 * nb + 1], alo, b2, b3);
+    }
+  }
+  __syncwarp();
+}
+
+template <bool V_F32>
+__global__ void __launch_bounds__(kWarps * 32, 2) skinny_mma_kernel(SkinnyArgs a) {
   constexpr int MT = 16;
   constexpr int COLS = kMmaCols;
   extern __shared__ __align__(16) float smem[];
@@ -215,84 +295,38 @@ __global__ void __launch_bounds__(kWarps * 32) skinny_mma_kernel(SkinnyArgs a) {
   const int kc = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(a.Kd - k0, a.k_chunk)));
   const int nvalid = static_cast<int>(std::min<int64_t>(COLS, a.Nd - n0));
 
-  float* sv = smem;                                         // [k_chunk][16] fp32
+  float* sv = smem;  // [k_chunk][16] fp32
   uint8_t* tbuf = reinterpret_cast<uint8_t*>(smem + a.k_chunk * MT) + warp * kMmaBufBytes;
   stage_v_kmajor<MT>(sv, a, k0, kc, a.k_chunk);
   __syncthreads();
 
-  float d[16][4];
+  float d[8][4];
 #pragma unroll
-  for (int t = 0; t < 16; ++t)
+  for (int t = 0; t < 8; ++t)
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[t][i] = 0.f;
 
-  const int half = lane >> 4;   // which of the two rows this lane loads
-  const int g16 = lane & 15;    // lane within the row
-  const int g = lane >> 2, tq = lane & 3;
-  const uint32_t tbase = smem_u32(tbuf);
-  // ldmatrix row address for this lane: matrix j = lane/8 covers rows
-  // (j&1)*8 .. +7 and columns (j>>1)*8 .. +7 of a 16×16 block.
-  const int lm_row = (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int lm_col = (lane >> 4) * 8;
-  const __nv_bfloat16* wbase = a.W + n0;
-
-  for (int ks = warp * 16; ks < kc; ks += kWarps * 16) {
-    // 1. 16 rows of W (realigned) into the warp buffer.
-    uint4 w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int k = ks + 2 * i + half;
-      const int nv = (k < kc) ? nvalid : 0;
-      w[i] = fetch_seg16(wbase + (k0 + k) * a.ldw, g16, 16, nv, a.w_lo, a.w_hi);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int row = 2 * i + half;
-      *reinterpret_cast<uint4*>(tbuf + row * kMmaRowBytes + g16 * 16) = w[i];
-    }
-    __syncwarp();
-    // 2. A fragment: tokens × 16 rows of W (k), from the staged V.
-    uint32_t ahi[4], alo[4];
-    {
-      const float* v0 = sv + (ks + 2 * tq) * MT;  // row k = ks + 2tq
-      const float* v1 = v0 + MT;                  // k + 1
-      const float* v8 = v0 + 8 * MT;              // k + 8
-      const float* v9 = v8 + MT;                  // k + 9
-      const float f[8] = {v0[g], v1[g], v0[g + 8], v1[g + 8], v8[g], v9[g], v8[g + 8], v9[g + 8]};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t h = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-        ahi[i] = h;
-        if (V_F32) {
-          const float r0 = f[2 * i] - bf16lo_to_f32(h);
-          const float r1 = f[2 * i + 1] - bf16hi_to_f32(h);
-          alo[i] = pack_bf16x2(r0, r1);
-        }
-      }
-    }
-    // 3. B fragments via ldmatrix.trans and the MMAs.
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_trans(tbase + lm_row * kMmaRowBytes + (nb * 16 + lm_col) * 2, b0, b1, b2, b3);
-      mma_bf16_16816(d[2 * nb], ahi, b0, b1);
-      mma_bf16_16816(d[2 * nb + 1], ahi, b2, b3);
-      if (V_F32) {
-        mma_bf16_16816(d[2 * nb], alo, b0, b1);
-        mma_bf16_16816(d[2 * nb + 1], alo, b2, b3);
-      }
-    }
-    __syncwarp();
+  MmaCtx c{a.W + n0, k0, a.ldw, kc, nvalid, a.w_lo, a.w_hi, lane >> 3, lane & 7};
+  uint4 ca[4], ea[4], cb[4], eb[4];
+  int ks = warp * 16;
+  mma_issue(c, ks, ca, ea);
+  mma_issue(c, ks + kMmaStep, cb, eb);
+  for (; ks < kc; ks += 2 * kMmaStep) {
+    mma_step<V_F32>(c, ks, ca, ea, tbuf, sv, d, lane);
+    mma_issue(c, ks + 2 * kMmaStep, ca, ea);
+    if (ks + kMmaStep < kc) mma_step<V_F32>(c, ks + kMmaStep, cb, eb, tbuf, sv, d, lane);
+    mma_issue(c, ks + 3 * kMmaStep, cb, eb);
   }
 
   // Per-warp partials: d[t] holds rows g, g+8 and columns 8t + 2tq, +1.
   __syncthreads();
   float* part = smem;  // [kWarps][16][COLS]
+  const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const int c = 8 * t + 2 * tq;
-    *reinterpret_cast<float2*>(part + (warp * MT + g) * COLS + c) = make_float2(d[t][0], d[t][1]);
-    *reinterpret_cast<float2*>(part + (warp * MT + g + 8) * COLS + c) =
+  for (int t = 0; t < 8; ++t) {
+    const int col = 8 * t + 2 * tq;
+    *reinterpret_cast<float2*>(part + (warp * MT + g) * COLS + col) = make_float2(d[t][0], d[t][1]);
+    *reinterpret_cast<float2*>(part + (warp * MT + g + 8) * COLS + col) =
         make_float2(d[t][2], d[t][3]);
   }
   reduce_and_finalise<MT, COLS>(a, part, n0, nvalid);
@@ -317,7 +351,7 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms) {
     p.cols = kMmaCols;
   }
   p.col_blocks = static_cast<int>((Nd + p.cols - 1) / p.cols);
-  const int ctas_per_sm = (p.kind == SkinnyKind::kFma) ? 4 : 2;
+  const int ctas_per_sm = 2;
   const int target = std::max(1, num_sms * ctas_per_sm);
   const int gran = (p.kind == SkinnyKind::kFma) ? kWarps : 16;
   int splits = std::max(1, (target + p.col_blocks - 1) / p.col_blocks);
@@ -325,7 +359,7 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms) {
   chunk = std::max<int64_t>(chunk, gran * 4);
   // Shared memory holds the CTA's slice of V: cap the row range so that two
   // (MMA) or four (FMA) CTAs still fit on an SM.
-  const int64_t cap = (p.kind == SkinnyKind::kFma) ? (24576 / p.mt) / gran * gran : 1216;
+  const int64_t cap = (p.kind == SkinnyKind::kFma) ? (24576 / p.mt) / gran * gran : 1024;
   chunk = std::min<int64_t>(chunk, cap);
   p.k_chunk = round_up(static_cast<int>(chunk), gran);
   p.splits = static_cast<int>((Kd + p.k_chunk - 1) / p.k_chunk);

@@ -18,7 +18,7 @@ namespace lr {
 
 __device__ __forceinline__ uint4 ld_nc_v4(uintptr_t a) {
   uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(a));
   return v;
@@ -26,14 +26,14 @@ __device__ __forceinline__ uint4 ld_nc_v4(uintptr_t a) {
 
 __device__ __forceinline__ uint2 ld_nc_v2(uintptr_t a) {
   uint2 v;
-  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(a));
+  asm("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(a));
   return v;
 }
 
 __device__ __forceinline__ uint32_t ld_u16_or0(uintptr_t p, uintptr_t lo, uintptr_t hi) {
   if (p < lo || p + 2 > hi) return 0u;
   unsigned short h;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(p));
+  asm("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(p));
   return h;
 }
 
@@ -75,6 +75,22 @@ __device__ __forceinline__ uint4 realign16(uint4 c, uint4 n, int s) {
     case 6: return make_uint4(c.w, n.x, n.y, n.z);
     default: return make_uint4(mid16(c.w, n.x), mid16(n.x, n.y), mid16(n.y, n.z), mid16(n.z, n.w));
   }
+}
+
+// The same without a branch on s, for groups narrower than a warp whose lanes
+// may hold rows with different shifts (a switch would diverge).
+__device__ __forceinline__ uint4 realign16_nb(uint4 c, uint4 n, int s) {
+  uint32_t w0 = c.x, w1 = c.y, w2 = c.z, w3 = c.w, w4 = n.x, w5 = n.y, w6 = n.z, w7 = n.w;
+  if (s & 4) {  // drop two words
+    w0 = w2; w1 = w3; w2 = w4; w3 = w5; w4 = w6; w5 = w7;
+  }
+  if (s & 2) {  // drop one word
+    w0 = w1; w1 = w2; w2 = w3; w3 = w4; w4 = w5;
+  }
+  if (s & 1) {  // drop one element
+    return make_uint4(mid16(w0, w1), mid16(w1, w2), mid16(w2, w3), mid16(w3, w4));
+  }
+  return make_uint4(w0, w1, w2, w3);
 }
 
 // Elements [s, s+4) of the 8-element concatenation (c, n), s in 0..3.
@@ -128,40 +144,43 @@ __device__ __forceinline__ uint2 mask_tail4(uint2 v, int keep) {
   return make_uint2(w[0], w[1]);
 }
 
-// One group of G lanes (g = lane index within the group, G a power of two
-// dividing 32) fetches a row segment that starts at element pointer p (2-byte
-// aligned): lane g returns elements [8g, 8g+8) of the segment, with elements
-// at index >= nvalid set to zero.  The shift must be the same for the whole
-// group, which holds because the group shares p.
-__device__ __forceinline__ uint4 fetch_seg16(const __nv_bfloat16* p, int g, int G, int nvalid,
-                                             uintptr_t lo, uintptr_t hi) {
+// Row-segment fetch, split in two so that many loads can be in flight before
+// the first one is consumed: seg16_issue() only loads, seg16_finish()
+// shuffles and realigns.  A group of G lanes (g = lane index within the
+// group, G a power of two dividing 32) fetches the segment that starts at
+// element pointer p (2-byte aligned): after finish, lane g holds elements
+// [8g, 8g+8) of it, with elements at index >= nvalid set to zero.  All lanes
+// of a group share p, hence the shift s = seg_shift(p).
+//   cur: aligned chunk g, i.e. segment elements [8g - s, 8g - s + 8)
+//   ext: (lane G-1 only) the chunk after the group's last one
+__device__ __forceinline__ int seg_shift(const __nv_bfloat16* p) {
+  return static_cast<int>((reinterpret_cast<uintptr_t>(p) & 15u) >> 1);
+}
+
+__device__ __forceinline__ void seg16_issue(const __nv_bfloat16* p, int g, int G, int nvalid,
+                                            uintptr_t lo, uintptr_t hi, uint4& cur, uint4& ext) {
   const uintptr_t a = reinterpret_cast<uintptr_t>(p);
   const uintptr_t base = a & ~static_cast<uintptr_t>(15);
   const int s = static_cast<int>((a & 15u) >> 1);
-  // Lane g's chunk holds segment elements [8g - s, 8g - s + 8): skip it when
-  // none of them is wanted.
+  // Fast path (the common case, decided once per group): the whole segment is
+  // wanted and every chunk the group touches lies inside the tensor.
+  if (nvalid >= 8 * G && base >= lo && base + 16u * (G + 1) <= hi) {
+    cur = ld_nc_v4(base + 16u * g);
+    ext = (g == G - 1 && s != 0) ? ld_nc_v4(base + 16u * G) : make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
   const bool need = nvalid > 0 && 8 * g - s < nvalid;
-  uint4 cur = need ? chunk16(base + 16u * g, lo, hi) : make_uint4(0u, 0u, 0u, 0u);
-  uint4 nxt = shfl_down_u4(cur, 1, G);
-  if (g == G - 1)
-    nxt = (s != 0 && 8 * G - s < nvalid) ? chunk16(base + 16u * G, lo, hi)
-                                         : make_uint4(0u, 0u, 0u, 0u);
-  uint4 v = realign16(cur, nxt, s);
-  return mask_tail8(v, nvalid - 8 * g);
+  cur = need ? chunk16(base + 16u * g, lo, hi) : make_uint4(0u, 0u, 0u, 0u);
+  ext = (g == G - 1 && s != 0 && 8 * G - s < nvalid) ? chunk16(base + 16u * G, lo, hi)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
 }
 
-__device__ __forceinline__ uint2 fetch_seg8(const __nv_bfloat16* p, int g, int G, int nvalid,
-                                            uintptr_t lo, uintptr_t hi) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-  const uintptr_t base = a & ~static_cast<uintptr_t>(7);
-  const int s = static_cast<int>((a & 7u) >> 1);
-  const bool need = nvalid > 0 && 4 * g - s < nvalid;
-  uint2 cur = need ? chunk8(base + 8u * g, lo, hi) : make_uint2(0u, 0u);
-  uint2 nxt = shfl_down_u2(cur, 1, G);
-  if (g == G - 1)
-    nxt = (s != 0 && 4 * G - s < nvalid) ? chunk8(base + 8u * G, lo, hi) : make_uint2(0u, 0u);
-  uint2 v = realign8(cur, nxt, s);
-  return mask_tail4(v, nvalid - 4 * g);
+__device__ __forceinline__ uint4 seg16_finish(uint4 cur, uint4 ext, int s, int g, int G,
+                                              int nvalid) {
+  uint4 nxt = shfl_down_u4(cur, 1, G);
+  if (g == G - 1) nxt = ext;
+  const uint4 v = (G == 32) ? realign16(cur, nxt, s) : realign16_nb(cur, nxt, s);
+  return (nvalid >= 8 * G) ? v : mask_tail8(v, nvalid - 8 * g);
 }
 
 }  // namespace lr

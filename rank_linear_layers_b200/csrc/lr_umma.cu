@@ -47,7 +47,8 @@ constexpr int EPI_WARPS = 4;
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
 constexpr int LOADER_WARP0 = 6;
-constexpr int LOADER_WARPS = 4;
+constexpr int LOADER_WARPS = 4;   // per loader group
+constexpr int LOADER_GROUPS = 2;  // groups take alternate k blocks
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
 constexpr unsigned kWhereProducer = 1, kWhereLoader = 2, kWhereMma = 3, kWhereMmaAcc = 4,
@@ -69,50 +70,63 @@ struct Smem {
 };
 
 // Manual (realigning) load of Aop's [128 × 64] K-major tile for k block kb.
-// Each loader warp fills 32 rows, four rows (8 lanes each) per instruction.
+// Each of the group's 4 loader warps fills 32 rows, four rows (8 lanes × 16 B
+// each) per instruction; all 8 instructions are issued before any is used.
 __device__ __forceinline__ void load_a_manual(uint8_t* dst, const GemmArgs& g, int m_blk, int kb,
                                               int lw, int lane) {
   const int gl = lane & 7;
   const int k0 = kb * BK;
   const int kvalid = min(BK, g.Kc - k0);
-  uint4 v[8];
+  uint4 cur[8], ext[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = lw * 32 + 4 * i + (lane >> 3);
     const int mg = m_blk * BM + m;
     const int nv = (mg < g.Mr) ? kvalid : 0;
-    v[i] = fetch_seg16(g.a + static_cast<int64_t>(mg) * g.lda + k0, gl, 8, nv, g.a_lo, g.a_hi);
+    seg16_issue(g.a + static_cast<int64_t>(mg) * g.lda + k0, gl, 8, nv, g.a_lo, g.a_hi, cur[i],
+                ext[i]);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = lw * 32 + 4 * i + (lane >> 3);
+    const int mg = m_blk * BM + m;
+    const int nv = (mg < g.Mr) ? kvalid : 0;
+    const uint4 v = seg16_finish(cur[i], ext[i], seg_shift(g.a + static_cast<int64_t>(mg) * g.lda + k0),
+                                 gl, 8, nv);
     uint8_t* p = dst + m * 128 + ((gl ^ (m & 7)) << 4);
-    *reinterpret_cast<uint4*>(p) = v[i];
+    *reinterpret_cast<uint4*>(p) = v;
   }
 }
 
-// Manual load of Bop's [64 × 256] MN-major tile: each loader warp fills 16
-// rows (k), one 512-byte row segment (32 lanes × 16 B) per instruction.
+// Manual load of Bop's [64 × 256] MN-major tile: each of the group's 4 loader
+// warps fills 16 rows (k), one 512-byte row segment (32 lanes × 16 B) per
+// instruction; all 16 are issued before any is used.
 __device__ __forceinline__ void load_b_manual(uint8_t* dst, const GemmArgs& g, int n_blk, int kb,
                                               int lw, int lane) {
   const int n0 = n_blk * BN;
   const int nvalid = min(BN, g.Nc - n0);
   constexpr int U = 8;
 #pragma unroll
-  for (int i0 = 0; i0 < 16; i0 += U) {
-    uint4 v[U];
+  for (int half = 0; half < 16 / U; ++half) {
+    uint4 cur[U], ext[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int k = lw + LOADER_WARPS * (i0 + u);
+      const int k = lw + LOADER_WARPS * (half * U + u);
       const int kg = kb * BK + k;
       const int nv = (kg < g.Kc) ? nvalid : 0;
-      v[u] = fetch_seg16(g.b + static_cast<int64_t>(kg) * g.ldb + n0, lane, 32, nv, g.b_lo, g.b_hi);
+      seg16_issue(g.b + static_cast<int64_t>(kg) * g.ldb + n0, lane, 32, nv, g.b_lo, g.b_hi,
+                  cur[u], ext[u]);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int k = lw + LOADER_WARPS * (i0 + u);
+      const int k = lw + LOADER_WARPS * (half * U + u);
+      const int kg = kb * BK + k;
+      const int nv = (kg < g.Kc) ? nvalid : 0;
+      const uint4 v = seg16_finish(cur[u], ext[u],
+                                   seg_shift(g.b + static_cast<int64_t>(kg) * g.ldb + n0), lane, 32,
+                                   nv);
       uint8_t* p = dst + (lane >> 3) * B_ATOM + k * 128 + (((lane & 7) ^ (k & 7)) << 4);
-      *reinterpret_cast<uint4*>(p) = v[u];
+      *reinterpret_cast<uint4*>(p) = v;
     }
   }
 }
@@ -152,7 +166,7 @@ template <bool A_TMA, bool B_TMA>
 struct GemmCfg {
   static constexpr bool kAnyManual = !A_TMA || !B_TMA;
   static constexpr bool kAnyTma = A_TMA || B_TMA;
-  static constexpr int kWarps = 6 + (kAnyManual ? LOADER_WARPS : 0);
+  static constexpr int kWarps = 6 + (kAnyManual ? LOADER_WARPS * LOADER_GROUPS : 0);
   static constexpr int kThreads = kWarps * 32;
 };
 
@@ -234,12 +248,17 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
       }
     }
   } else if (Cfg::kAnyManual && warp >= LOADER_WARP0) {
-    const int lw = warp - LOADER_WARP0;
-    int s = 0;
-    uint32_t ph = 0;
+    // Loader group lg takes every LOADER_GROUPS-th k block of the flattened
+    // (tile, k block) sequence, so two stages fill concurrently.
+    const int lw = (warp - LOADER_WARP0) % LOADER_WARPS;
+    const int lg = (warp - LOADER_WARP0) / LOADER_WARPS;
+    int q = 0;  // index in the flattened (tile, k block) sequence
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = 0; kb < num_kb; ++kb, ++q) {
+        if (q % LOADER_GROUPS != lg) continue;
+        const int s = q % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(q / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereLoader)) {
           ok = false;
           break;
@@ -249,10 +268,6 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
     }
   } else if (warp == MMA_WARP) {
