@@ -267,21 +267,18 @@ lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const vo
   return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias);
 }
 
+bool tma_ok(const void* p, int64_t ld) {
+  return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && (ld % 8 == 0);
+}
+
+// One prefill GEMM: C = a · b (+bias), both operands already TMA-able.
 lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, const void* b,
                int64_t ldb, void* c, int64_t ldc, const void* bias, int64_t Mr, int64_t Nc,
-               int64_t Kc, size_t a_bytes, size_t b_bytes) {
+               int64_t Kc) {
   GemmArgs g{};
   g.Mr = static_cast<int>(Mr);
   g.Nc = static_cast<int>(Nc);
   g.Kc = static_cast<int>(Kc);
-  g.a = static_cast<const __nv_bfloat16*>(a);
-  g.lda = lda;
-  g.a_lo = reinterpret_cast<uintptr_t>(a);
-  g.a_hi = g.a_lo + a_bytes;
-  g.b = static_cast<const __nv_bfloat16*>(b);
-  g.ldb = ldb;
-  g.b_lo = reinterpret_cast<uintptr_t>(b);
-  g.b_hi = g.b_lo + b_bytes;
   g.c = static_cast<__nv_bfloat16*>(c);
   g.ldc = ldc;
   g.bias = static_cast<const __nv_bfloat16*>(bias);
@@ -289,32 +286,61 @@ lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, c
   g.tiles_n = static_cast<int>((Nc + kGemmBN - 1) / kGemmBN);
   g.wait = wait_ctl(d);
   GemmMaps maps{};
-  maps.a_tma = (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (lda % 8 == 0);
-  maps.b_tma = (reinterpret_cast<uintptr_t>(b) % 16 == 0) && (ldb % 8 == 0);
-  if (maps.a_tma) {
-    lr_status st = tensor_map(&maps.a, a, Kc, Mr, lda, kGemmBK, kGemmBM);
-    if (st != LR_OK) return st;
-  }
-  if (maps.b_tma) {
-    lr_status st = tensor_map(&maps.b, b, Nc, Kc, ldb, 64, kGemmBK);
-    if (st != LR_OK) return st;
-  }
+  lr_status st = tensor_map(&maps.a, a, Kc, Mr, lda, kGemmBK, kGemmBM);
+  if (st != LR_OK) return st;
+  st = tensor_map(&maps.b, b, Nc, Kc, ldb, 64, kGemmBK);
+  if (st != LR_OK) return st;
   return launched(launch_gemm(g, maps, d->sms, stream));
+}
+
+// A TMA-able view of a [rows, cols] operand: itself, or a realigned copy in
+// `scratch` (advanced past the copy).
+struct Operand {
+  const void* p;
+  int64_t ld;
+};
+
+size_t repack_bytes(const void* p, int64_t ld, int64_t rows, int64_t cols) {
+  if (tma_ok(p, ld) || rows == 0 || cols == 0) return 0;
+  return align_up(static_cast<size_t>(rows) * align_up(static_cast<size_t>(cols), 8) * 2, 256);
+}
+
+lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t ld, int64_t rows,
+                      int64_t cols, char** scratch, Operand* out) {
+  if (tma_ok(p, ld)) {
+    *out = Operand{p, ld};
+    return LR_OK;
+  }
+  const int64_t ldd = static_cast<int64_t>(align_up(static_cast<size_t>(cols), 8));
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(*scratch);
+  *scratch += repack_bytes(p, ld, rows, cols);
+  lr_status st = launched(launch_repack(static_cast<const __nv_bfloat16*>(p), ld,
+                                        span_bytes(rows, cols, ld), dst, ldd, rows, cols, d->sms,
+                                        stream));
+  if (st != LR_OK) return st;
+  *out = Operand{dst, ldd};
+  return LR_OK;
 }
 
 lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                       const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
                       int64_t N, int64_t ldy) {
   const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), 8));
+  const size_t tbytes = align_up(static_cast<size_t>(M) * ldt * 2, 256);
+  const size_t need = tbytes + repack_bytes(X, K, M, K) + repack_bytes(A, r, K, r) +
+                      repack_bytes(B, N, r, N);
   char *zero = nullptr, *scratch = nullptr;
-  lr_status st = workspace(stream, 0, static_cast<size_t>(M) * ldt * 2, &zero, &scratch);
+  lr_status st = workspace(stream, 0, need, &zero, &scratch);
   if (st != LR_OK) return st;
   void* T = scratch;
-  st = gemm(d, stream, X, K, A, r, T, ldt, nullptr, M, r, K, span_bytes(M, K, K),
-            span_bytes(K, r, r));
+  scratch += tbytes;
+  Operand x, a, b;
+  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b)) != LR_OK) return st;
+  st = gemm(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K);
   if (st != LR_OK) return st;
-  return gemm(d, stream, T, ldt, B, N, Y, ldy, bias, M, N, r, span_bytes(M, r, ldt),
-              span_bytes(r, N, N));
+  return gemm(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r);
 }
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
@@ -489,8 +515,16 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
     return skinny(d, stream, m, X, K, false, W, K, N, reinterpret_cast<float*>(zero),
                   reinterpret_cast<unsigned int*>(zero + acc), nullptr, 0, Y, N, bias);
   }
-  return gemm(d, stream, X, K, W, N, Y, N, bias, M, N, K, span_bytes(M, K, K),
-              span_bytes(K, N, N));
+  {
+    const size_t need = repack_bytes(X, K, M, K) + repack_bytes(W, N, K, N);
+    char *zero = nullptr, *scratch = nullptr;
+    st = workspace(stream, 0, need, &zero, &scratch);
+    if (st != LR_OK) return st;
+    Operand x, w;
+    if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x)) != LR_OK) return st;
+    if ((st = tma_operand(d, stream, W, N, K, N, &scratch, &w)) != LR_OK) return st;
+    return gemm(d, stream, x.p, x.ld, w.p, w.ld, Y, N, bias, M, N, K);
+  }
 }
 
 lr_status lr_last_device_status(void* stream) {

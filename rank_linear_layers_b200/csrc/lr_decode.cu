@@ -351,18 +351,31 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms) {
     p.cols = kMmaCols;
   }
   p.col_blocks = static_cast<int>((Nd + p.cols - 1) / p.cols);
-  const int ctas_per_sm = 2;
-  const int target = std::max(1, num_sms * ctas_per_sm);
+  // Split W's rows so that the grid fills the resident CTA slots in whole
+  // waves: the cost of a split count is (waves × rows per CTA), scaled up
+  // when the grid leaves slots empty, plus a small charge per split for the
+  // partial-sum atomics.
+  const int capacity = std::max(1, num_sms * 2);
   const int gran = (p.kind == SkinnyKind::kFma) ? kWarps : 16;
-  int splits = std::max(1, (target + p.col_blocks - 1) / p.col_blocks);
-  int64_t chunk = (Kd + splits - 1) / splits;
-  chunk = std::max<int64_t>(chunk, gran * 4);
-  // Shared memory holds the CTA's slice of V: cap the row range so that two
-  // (MMA) or four (FMA) CTAs still fit on an SM.
   const int64_t cap = (p.kind == SkinnyKind::kFma) ? (24576 / p.mt) / gran * gran : 1024;
-  chunk = std::min<int64_t>(chunk, cap);
-  p.k_chunk = round_up(static_cast<int>(chunk), gran);
+  const int64_t max_splits = std::max<int64_t>(1, std::min<int64_t>(512, (Kd + gran - 1) / gran));
+  double best = 1e300;
+  p.k_chunk = static_cast<int>(std::min<int64_t>(cap, round_up(static_cast<int>(std::min<int64_t>(Kd, 1 << 30)), gran)));
   p.splits = static_cast<int>((Kd + p.k_chunk - 1) / p.k_chunk);
+  for (int64_t sp = 1; sp <= max_splits; ++sp) {
+    int64_t chunk = (Kd + sp - 1) / sp;
+    chunk = std::min<int64_t>(cap, (chunk + gran - 1) / gran * gran);
+    const int64_t splits = (Kd + chunk - 1) / chunk;
+    const int64_t items = splits * p.col_blocks;
+    const int64_t waves = (items + capacity - 1) / capacity;
+    const double fill = static_cast<double>(std::min<int64_t>(items, capacity)) / capacity;
+    const double cost = static_cast<double>(waves * chunk) / fill + 0.5 * static_cast<double>(splits);
+    if (cost < best) {
+      best = cost;
+      p.k_chunk = static_cast<int>(chunk);
+      p.splits = static_cast<int>(splits);
+    }
+  }
   if (p.splits < 1) p.splits = 1;
   const size_t stage = static_cast<size_t>(p.k_chunk) * p.mt * sizeof(float);
   const size_t part = static_cast<size_t>(kWarps) * p.mt * p.cols * sizeof(float);

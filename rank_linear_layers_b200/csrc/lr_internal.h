@@ -58,15 +58,12 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& args, cudaSt
 
 // ------------------------------------------------------------------ prefill
 // C[Mr, Nc] = Aop[Mr, Kc] · Bop[Kc, Nc] (+ bias), bf16 in, fp32 accumulate,
-// bf16 out.  Aop is row-major (K contiguous), Bop is row-major (N contiguous).
+// bf16 out.  Aop is row-major (K contiguous), Bop is row-major (N
+// contiguous); both are read through TMA tensor maps, so their base
+// addresses and row pitches must be 16-byte aligned.  C may have any
+// 2-byte-aligned base and pitch.
 struct GemmArgs {
   int Mr, Nc, Kc;
-  const __nv_bfloat16* a;
-  int64_t lda;
-  uintptr_t a_lo, a_hi;
-  const __nv_bfloat16* b;
-  int64_t ldb;
-  uintptr_t b_lo, b_hi;
   __nv_bfloat16* c;
   int64_t ldc;
   const __nv_bfloat16* bias;
@@ -75,9 +72,8 @@ struct GemmArgs {
 };
 
 struct GemmMaps {
-  CUtensorMap a;  // valid when a_tma
-  CUtensorMap b;  // valid when b_tma
-  bool a_tma, b_tma;
+  CUtensorMap a;  // Aop: dims {Kc, Mr}, box {64, 128}
+  CUtensorMap b;  // Bop: dims {Nc, Kc}, box {64, 64}
 };
 
 constexpr int kGemmBM = 128;
@@ -88,6 +84,12 @@ constexpr int kGemmStages = 4;
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm(const GemmArgs& args, const GemmMaps& maps, int num_sms,
                         cudaStream_t stream);
+
+// Copy a [rows, cols] bf16 matrix with any 2-byte-aligned base and pitch lds
+// into dst (16-byte-aligned base, pitch ldd >= cols rounded up to 8).
+cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_bytes,
+                          __nv_bfloat16* dst, int64_t ldd, int64_t rows, int64_t cols,
+                          int num_sms, cudaStream_t stream);
 
 // Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0).
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,

@@ -8,28 +8,25 @@
 // Bop row-major (N contiguous: "MN-major"); the tensor core reads both
 // layouts from shared memory directly, so no operand is transposed.
 //
-// Structure (one persistent CTA per SM, warp-specialised):
+// Structure (one persistent CTA per SM, warp-specialised, 192 threads):
 //   warps 0-3  epilogue: TMEM -> registers -> +bias -> bf16 -> global
 //   warp 4     one elected thread issues tcgen05.mma (128×256×16 per issue)
-//   warp 5     one thread issues TMA tile loads for operands whose row
-//              stride is a multiple of 16 bytes (TMA's requirement)
-//   warps 6-9  (only when an operand's row stride is not a multiple of 16
-//              bytes, e.g. A [K, r] with odd r) realigning loaders that write
-//              the same 128-byte-swizzled layout TMA would
+//   warp 5     one thread issues the TMA tile loads (128-byte swizzle)
 // A 4-stage shared-memory ring (mbarrier full/empty pairs) feeds the MMA;
 // two TMEM accumulators (2 × 256 fp32 columns) let the epilogue of one tile
-// overlap the main loop of the next.
+// overlap the main loop of the next.  Operands must have 16-byte-aligned
+// bases and row pitches (TMA's rule); the host realigns any that do not
+// (lr_repack.cu) before launching.
 //
 // Ragged edges cost no padding on the host: TMA zero-fills out-of-bounds
-// rows and columns, the loaders zero them, the last K block issues only the
-// 16-deep MMA steps it needs, and the epilogue predicates rows and columns.
-// This is the point of the GAC paper's §3 analysis (misaligned K or N fall to
-// slower library kernels and partially filled tensor-core tiles): here a
-// misaligned r changes the loader, not the tile shape or the MMA rate.
+// rows and columns, the last K block issues only the 16-deep MMA steps it
+// needs, and the epilogue predicates rows and columns.  This is the point of
+// the GAC paper's §3 analysis (misaligned K or N fall to slower library
+// kernels and partially filled tensor-core tiles): here a misaligned r
+// changes neither the tile shape nor the MMA rate.
 #include <algorithm>
 
 #include "lr_internal.h"
-#include "lr_load.cuh"
 
 namespace lr {
 
@@ -46,13 +43,9 @@ constexpr int B_ATOM = BK * 128;      // one 64-column MN-major atom column: 8 K
 constexpr int EPI_WARPS = 4;
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
-constexpr int LOADER_WARP0 = 6;
-constexpr int LOADER_WARPS = 4;   // per loader group
-constexpr int LOADER_GROUPS = 2;  // groups take alternate k blocks
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
-constexpr unsigned kWhereProducer = 1, kWhereLoader = 2, kWhereMma = 3, kWhereMmaAcc = 4,
-                   kWhereEpilogue = 5;
+constexpr unsigned kWhereProducer = 1, kWhereMma = 3, kWhereMmaAcc = 4, kWhereEpilogue = 5;
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
                                                 unsigned long long limit_ns) {
@@ -68,68 +61,6 @@ struct Smem {
   __device__ uint8_t* a(int s) const { return base + s * STAGE; }
   __device__ uint8_t* b(int s) const { return base + s * STAGE + A_STAGE; }
 };
-
-// Manual (realigning) load of Aop's [128 × 64] K-major tile for k block kb.
-// Each of the group's 4 loader warps fills 32 rows, four rows (8 lanes × 16 B
-// each) per instruction; all 8 instructions are issued before any is used.
-__device__ __forceinline__ void load_a_manual(uint8_t* dst, const GemmArgs& g, int m_blk, int kb,
-                                              int lw, int lane) {
-  const int gl = lane & 7;
-  const int k0 = kb * BK;
-  const int kvalid = min(BK, g.Kc - k0);
-  uint4 cur[8], ext[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int m = lw * 32 + 4 * i + (lane >> 3);
-    const int mg = m_blk * BM + m;
-    const int nv = (mg < g.Mr) ? kvalid : 0;
-    seg16_issue(g.a + static_cast<int64_t>(mg) * g.lda + k0, gl, 8, nv, g.a_lo, g.a_hi, cur[i],
-                ext[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int m = lw * 32 + 4 * i + (lane >> 3);
-    const int mg = m_blk * BM + m;
-    const int nv = (mg < g.Mr) ? kvalid : 0;
-    const uint4 v = seg16_finish(cur[i], ext[i], seg_shift(g.a + static_cast<int64_t>(mg) * g.lda + k0),
-                                 gl, 8, nv);
-    uint8_t* p = dst + m * 128 + ((gl ^ (m & 7)) << 4);
-    *reinterpret_cast<uint4*>(p) = v;
-  }
-}
-
-// Manual load of Bop's [64 × 256] MN-major tile: each of the group's 4 loader
-// warps fills 16 rows (k), one 512-byte row segment (32 lanes × 16 B) per
-// instruction; all 16 are issued before any is used.
-__device__ __forceinline__ void load_b_manual(uint8_t* dst, const GemmArgs& g, int n_blk, int kb,
-                                              int lw, int lane) {
-  const int n0 = n_blk * BN;
-  const int nvalid = min(BN, g.Nc - n0);
-  constexpr int U = 8;
-#pragma unroll
-  for (int half = 0; half < 16 / U; ++half) {
-    uint4 cur[U], ext[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = lw + LOADER_WARPS * (half * U + u);
-      const int kg = kb * BK + k;
-      const int nv = (kg < g.Kc) ? nvalid : 0;
-      seg16_issue(g.b + static_cast<int64_t>(kg) * g.ldb + n0, lane, 32, nv, g.b_lo, g.b_hi,
-                  cur[u], ext[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = lw + LOADER_WARPS * (half * U + u);
-      const int kg = kb * BK + k;
-      const int nv = (kg < g.Kc) ? nvalid : 0;
-      const uint4 v = seg16_finish(cur[u], ext[u],
-                                   seg_shift(g.b + static_cast<int64_t>(kg) * g.ldb + n0), lane, 32,
-                                   nv);
-      uint8_t* p = dst + (lane >> 3) * B_ATOM + k * 128 + (((lane & 7) ^ (k & 7)) << 4);
-      *reinterpret_cast<uint4*>(p) = v;
-    }
-  }
-}
 
 __device__ __forceinline__ void store_chunk(const GemmArgs& g, int row, int col0,
                                             const uint32_t (&v)[32], bool vec_ok) {
@@ -162,19 +93,11 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int row, int col0
   }
 }
 
-template <bool A_TMA, bool B_TMA>
-struct GemmCfg {
-  static constexpr bool kAnyManual = !A_TMA || !B_TMA;
-  static constexpr bool kAnyTma = A_TMA || B_TMA;
-  static constexpr int kWarps = 6 + (kAnyManual ? LOADER_WARPS * LOADER_GROUPS : 0);
-  static constexpr int kThreads = kWarps * 32;
-};
+constexpr int kGemmThreads = 6 * 32;
 
-template <bool A_TMA, bool B_TMA>
-__global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                      const __grid_constant__ CUtensorMap map_b, const GemmArgs g) {
-  using Cfg = GemmCfg<A_TMA, B_TMA>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   Smem sm{smem_raw + (((raw + 1023u) & ~1023u) - raw)};
@@ -190,7 +113,7 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], (Cfg::kAnyTma ? 1u : 0u) + (Cfg::kAnyManual ? LOADER_WARPS : 0u));
+      mbar_init(&full[s], 1u);
       mbar_init(&empty[s], 1u);
     }
     for (int i = 0; i < 2; ++i) {
@@ -205,8 +128,8 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
     tmem_relinquish();
   }
   if (warp == TMA_WARP && lane == 0) {
-    if (A_TMA) tma_prefetch_desc(&map_a);
-    if (B_TMA) tma_prefetch_desc(&map_b);
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
   }
   tc_fence_before();
   __syncthreads();
@@ -222,7 +145,7 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
   bool ok = true;
 
   if (warp == TMA_WARP) {
-    if (Cfg::kAnyTma && lane == 0) {
+    if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -232,42 +155,17 @@ __global__ void __launch_bounds__(GemmCfg<A_TMA, B_TMA>::kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], (A_TMA ? A_STAGE : 0) + (B_TMA ? B_STAGE : 0));
-          if (A_TMA) tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
-          if (B_TMA) {
+          mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
+          tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
-          }
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
           issued_phase[s] = static_cast<int>(ph);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
-      }
-    }
-  } else if (Cfg::kAnyManual && warp >= LOADER_WARP0) {
-    // Loader group lg takes every LOADER_GROUPS-th k block of the flattened
-    // (tile, k block) sequence, so two stages fill concurrently.
-    const int lw = (warp - LOADER_WARP0) % LOADER_WARPS;
-    const int lg = (warp - LOADER_WARP0) / LOADER_WARPS;
-    int q = 0;  // index in the flattened (tile, k block) sequence
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
-      for (int kb = 0; kb < num_kb; ++kb, ++q) {
-        if (q % LOADER_GROUPS != lg) continue;
-        const int s = q % STAGES;
-        const uint32_t ph = static_cast<uint32_t>(q / STAGES) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereLoader)) {
-          ok = false;
-          break;
-        }
-        if (!A_TMA) load_a_manual(sm.a(s), g, m_blk, kb, lw, lane);
-        if (!B_TMA) load_b_manual(sm.b(s), g, n_blk, kb, lw, lane);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
       }
     }
   } else if (warp == MMA_WARP) {
@@ -371,20 +269,6 @@ __global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64
   }
 }
 
-template <bool A_TMA, bool B_TMA>
-cudaError_t launch_impl(const GemmArgs& g, const GemmMaps& maps, int num_sms,
-                        cudaStream_t stream) {
-  using Cfg = GemmCfg<A_TMA, B_TMA>;
-  auto kern = umma_gemm_kernel<A_TMA, B_TMA>;
-  const size_t smem = gemm_smem_bytes();
-  cudaError_t e = ensure_max_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int tiles = g.tiles_m * g.tiles_n;
-  const int grid = std::max(1, std::min(tiles, num_sms));
-  kern<<<grid, Cfg::kThreads, smem, stream>>>(maps.a, maps.b, g);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 size_t gemm_smem_bytes() {
@@ -393,10 +277,14 @@ size_t gemm_smem_bytes() {
 
 cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,
                         cudaStream_t stream) {
-  if (maps.a_tma && maps.b_tma) return launch_impl<true, true>(g, maps, num_sms, stream);
-  if (maps.a_tma) return launch_impl<true, false>(g, maps, num_sms, stream);
-  if (maps.b_tma) return launch_impl<false, true>(g, maps, num_sms, stream);
-  return launch_impl<false, false>(g, maps, num_sms, stream);
+  const size_t smem = gemm_smem_bytes();
+  cudaError_t e =
+      ensure_max_smem(reinterpret_cast<const void*>(umma_gemm_kernel), static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int tiles = g.tiles_m * g.tiles_n;
+  const int grid = std::max(1, std::min(tiles, num_sms));
+  umma_gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(maps.a, maps.b, g);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
