@@ -116,6 +116,34 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
                    int64_t N, void* stream);
 
 /*
+ * lr_linear_decode_static — the decode path of lr_linear (M <= 16) for callers
+ * that cannot let a library allocate device memory: a serving loop with a
+ * hard latency budget (cudaMalloc/cudaFree synchronise the whole device), or
+ * a host application whose own pool allocator owns all device memory.  The
+ * paper has no counterpart to this entry point; it exists for such callers.
+ *
+ * Arguments and result are those of lr_linear (device pointers, bf16,
+ * row-major; asynchronous on `stream`).  The caller still provides X, A, B,
+ * bias and Y.  All scratch (partial sums, counters, T = X·A in fp32, about
+ * 1.6 MB) is one fixed array compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  Never calls cudaMalloc,
+ * cudaFree or any allocating library routine.
+ *
+ * Limits: M <= 16, r <= 4096, N <= 16384 (K < 2^31).  Larger sizes return
+ * LR_ERR_UNSUPPORTED without launching anything.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call clears the parts of the array that
+ * must start at zero.  All calls on a device share the array: calls whose
+ * kernels overlap on the GPU (on different streams or host threads) race and
+ * give wrong results; order them on one stream.
+ */
+lr_status lr_linear_decode_static(const void* X, const void* A, const void* B, const void* bias,
+                                  void* Y, int64_t M, int64_t K, int64_t r, int64_t N,
+                                  void* stream);
+
+/*
  * lr_last_device_status — synchronises `stream`, then reports and clears the
  * device status word of the current device: LR_ERR_TIMEOUT if a bounded
  * device-side wait ran out since the last call, else LR_OK.  After a timeout

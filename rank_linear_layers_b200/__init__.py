@@ -31,7 +31,7 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 EXPORTS = (
     "lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense", "lr_last_device_status",
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
-    "lr_kernel_launch_count", "lr_release_workspaces",
+    "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
 )
 
 
@@ -68,6 +68,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_linear_group.argtypes = [ctypes.POINTER(LrProj), ctypes.c_int, i64, vp]
     L.lr_linear_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_dense.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+    L.lr_linear_decode_static.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_last_device_status.argtypes = [vp]
     L.lr_status_string.argtypes = [ctypes.c_int]
     L.lr_status_string.restype = ctypes.c_char_p
@@ -78,6 +79,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
     for name in ("lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense",
+                 "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces"):
         getattr(L, name).restype = ctypes.c_int

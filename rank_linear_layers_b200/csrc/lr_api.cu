@@ -388,6 +388,10 @@ bool y_disjoint(const lr_proj& p, const lr_proj& q, int64_t M) {
 
 }  // namespace
 
+void note_cuda_error(int e) { g_last_cuda_error = e; }
+
+void note_launches(int n) { g_launches += n; }
+
 cudaError_t ensure_max_smem(const void* kernel, int bytes) {
   static std::mutex mu;
   static std::set<std::tuple<const void*, int, int>> done;

@@ -10,6 +10,11 @@
 
 namespace lr {
 
+// Record a CUDA error for lr_last_cuda_error(), and count kernel launches
+// for lr_kernel_launch_count(), from entry points outside lr_api.cu.
+void note_cuda_error(int e);
+void note_launches(int n);
+
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
 cudaError_t ensure_max_smem(const void* kernel, int bytes);
 
