@@ -236,6 +236,7 @@ lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64
   a.out_bf16 = static_cast<__nv_bfloat16*>(out_bf16);
   a.ld_out = ld_out;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
+  a.wait = wait_ctl(d);
   return launched(launch_skinny(plan, a, stream));
 }
 
@@ -540,6 +541,10 @@ lr_status lr_last_device_status(void* stream) {
   if (st != LR_OK) return st;
   DevStatus h{};
   LR_CUDA(cudaMemcpy(&h, d->status, sizeof h, cudaMemcpyDeviceToHost));
+  // The allocation-free entry point keeps its own status word.
+  unsigned int static_code = 0;
+  LR_CUDA(static_status_take(&static_code));
+  h.code |= static_code;
   if (h.code == 0 && h.abort == 0) return LR_OK;
   LR_CUDA(cudaMemset(d->status, 0, sizeof(DevStatus)));
   return (h.code & LR_DEV_TIMEOUT) ? LR_ERR_TIMEOUT : LR_ERR_CUDA;

@@ -53,7 +53,6 @@ constexpr int kMmaRowBytes = 8 * 16 + 16;  // 8 chunks per warp row, padded for 
 constexpr int kMmaBufBytes = 16 * kMmaRowBytes;
 constexpr int kMmaInflight = 3;  // k-steps whose loads are in flight per warp
 
-int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 constexpr int kSkinnyMaxSmem = 200 * 1024;
 

@@ -15,6 +15,10 @@ namespace lr {
 void note_cuda_error(int e);
 void note_launches(int n);
 
+// Read and clear the status word of lr_linear_decode_static on the current
+// device (0 if that entry point was never used there).  Allocates nothing.
+cudaError_t static_status_take(unsigned int* code);
+
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
 cudaError_t ensure_max_smem(const void* kernel, int bytes);
 
@@ -43,6 +47,7 @@ struct SkinnyArgs {
   __nv_bfloat16* out_bf16;  // else bf16 result (+bias) [M, ld_out]
   int64_t ld_out;
   const __nv_bfloat16* bias;
+  WaitCtl wait;             // bounded waits on the copy pipeline
 };
 
 enum class SkinnyKind { kFma, kMma };

@@ -31,7 +31,8 @@ constexpr size_t kAcc1Bytes = kStaticMaxM * kStaticMaxR * 4;   // phase-1 partia
 constexpr size_t kAcc2Bytes = kStaticMaxM * kStaticMaxN * 4;   // phase-2 partial sums
 constexpr size_t kCtrBytes = 2 * kStaticMaxCounters * 4;        // last-CTA counters
 constexpr size_t kTBytes = kStaticMaxM * kStaticMaxR * 4;      // T = X·A in fp32
-constexpr size_t kStaticBytes = kAcc1Bytes + kAcc2Bytes + kCtrBytes + kTBytes;  // ~1.6 MB
+constexpr size_t kStatusBytes = 256;                            // device status word
+constexpr size_t kStaticBytes = kAcc1Bytes + kAcc2Bytes + kCtrBytes + kTBytes + kStatusBytes;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 
@@ -81,6 +82,27 @@ bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
 }
 
 }  // namespace
+
+cudaError_t static_status_take(unsigned int* code) {
+  *code = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (dev < 0 || dev >= kMaxDevices || !g_static_ptr[dev]) return cudaSuccess;
+    base = g_static_ptr[dev];
+  }
+  DevStatus* st = reinterpret_cast<DevStatus*>(base + kStaticBytes - kStatusBytes);
+  DevStatus h{};
+  e = cudaMemcpy(&h, st, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return e;
+  if (h.code || h.abort) e = cudaMemset(st, 0, sizeof(DevStatus));
+  *code = h.code;
+  return e;
+}
+
 }  // namespace lr
 
 using namespace lr;
@@ -131,6 +153,9 @@ extern "C" lr_status lr_linear_decode_static(const void* X, const void* A, const
 
   SkinnyArgs a{};
   a.M = m;
+  // Bounded waits report to a status word kept in the same array.
+  a.wait = WaitCtl{reinterpret_cast<DevStatus*>(scratch + kStaticBytes - kStatusBytes),
+                   2000000000ull};
   // Phase 1: T = X·A (fp32).
   a.Kd = K;
   a.Nd = r;
