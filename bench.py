@@ -363,6 +363,12 @@ def run_ours(args):
                 "algorithmic_bytes_per_step": acc.algorithmic_bytes(M, K, R, N),
                 "flops_per_step": fl_step}
 
+    if args.profile:
+        # Prefill steps only, for ncu captures of this command.
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": ms, "gpu_launches": int(launches_timed)}))
+        return 0
+
     # End to end through the host-buffer C ABI call (pinned host memory).
     e2e = None
     try:
@@ -432,6 +438,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only the timed prefill steps (for ncu captures); numbers are not a bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
