@@ -160,7 +160,9 @@ int lr_last_cuda_error(void);
 /*
  * lr_set_path — testing and benchmarking control of the dispatch:
  *   0 = automatic (M <= 16 decode, else prefill), 1 = force decode (M <= 16
- *   only; larger M returns LR_ERR_INVALID_ARG), 2 = force prefill.
+ *   only; larger M returns LR_ERR_INVALID_ARG), 2 = force prefill, 3 = force
+ *   prefill on single-SM tiles (the default prefill kernel), 4 = force prefill
+ *   on CTA pairs (2-SM MMA, 256×256 tiles; M <= 128 still uses single SMs).
  * lr_set_wait_limit_ns — time limit of every device-side bounded wait
  *   (default 2e9 ns); 0 restores the default.
  * Both are process-wide and take effect on the next call.

@@ -25,7 +25,7 @@ LR_ERR_CUDA = 3
 LR_ERR_TIMEOUT = 4
 LR_ERR_NO_MEMORY = 5
 
-PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_PREFILL_1SM, PATH_PREFILL_PAIR = 0, 1, 2, 3, 4
 
 # Every symbol include/lr_linear.h declares.
 EXPORTS = (

@@ -215,7 +215,7 @@ lr_status launched(cudaError_t e, int n = 1) {
 lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64_t ldv, bool v_f32,
                  const void* W, int64_t Kd, int64_t Nd, float* acc, unsigned int* counters,
                  float* out_f32, int64_t ld_out_f32, void* out_bf16, int64_t ld_out,
-                 const void* bias) {
+                 const void* bias, bool dependent = false) {
   const SkinnyPlan plan = plan_skinny(M, Kd, Nd, d->sms);
   SkinnyArgs a{};
   a.M = M;
@@ -237,7 +237,7 @@ lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64
   a.ld_out = ld_out;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.wait = wait_ctl(d);
-  return launched(launch_skinny(plan, a, stream));
+  return launched(launch_skinny(plan, a, stream, dependent));
 }
 
 size_t acc_bytes(int M, int64_t n) { return align_up(static_cast<size_t>(M) * align_up(n, 4) * 4, 256); }
@@ -265,7 +265,9 @@ lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const vo
   // Phase 1: T = X·A (fp32).  Phase 2: Y = T·B + bias.
   st = skinny(d, stream, m, X, K, false, A, K, r, a1, k1, T, ldt, nullptr, 0, nullptr);
   if (st != LR_OK) return st;
-  return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias);
+  // Phase 2 starts streaming B while phase 1 finishes (programmatic
+  // dependent launch); it reads T only after phase 1 has completed.
+  return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias, true);
 }
 
 bool tma_ok(const void* p, int64_t ld) {
@@ -291,6 +293,9 @@ lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, c
   if (st != LR_OK) return st;
   st = tensor_map(&maps.b, b, Nc, Kc, ldb, 64, kGemmBK);
   if (st != LR_OK) return st;
+  // Single-SM tiles by default; CTA pairs (2-SM MMA, 256-row tiles) when
+  // selected with lr_set_path(4) (measured no faster on the prefill shapes).
+  if (Mr > kGemmBM && g_path.load() == 4) return launched(launch_gemm_pair(g, maps, d->sms, stream));
   return launched(launch_gemm(g, maps, d->sms, stream));
 }
 
@@ -565,7 +570,7 @@ const char* lr_status_string(lr_status s) {
 int lr_last_cuda_error(void) { return g_last_cuda_error; }
 
 lr_status lr_set_path(int path) {
-  if (path < 0 || path > 2) return LR_ERR_INVALID_ARG;
+  if (path < 0 || path > 4) return LR_ERR_INVALID_ARG;
   g_path.store(path);
   return LR_OK;
 }

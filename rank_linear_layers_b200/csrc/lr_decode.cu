@@ -108,7 +108,7 @@ __device__ __forceinline__ void reduce_and_finalise(const SkinnyArgs& a, const f
 
 __device__ __forceinline__ float load_v(const SkinnyArgs& a, int m, int64_t k) {
   const int64_t idx = static_cast<int64_t>(m) * a.ldv + k;
-  return a.v_f32 ? __ldg(static_cast<const float*>(a.V) + idx)
+  return a.v_f32 ? __ldcg(static_cast<const float*>(a.V) + idx)
                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.V)[idx]);
 }
 
@@ -121,19 +121,12 @@ __global__ void __launch_bounds__(kFmaWarps * 32, 2) skinny_fma_kernel(SkinnyArg
   extern __shared__ __align__(16) float smem[];
   float2* sv2 = reinterpret_cast<float2*>(smem);             // [k_chunk][MT]
   float* part = smem + 2 * a.k_chunk * MT;                   // [MT][CB]
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * CB;
   const int64_t k0 = static_cast<int64_t>(blockIdx.y) * a.k_chunk;
   const int kc = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(a.Kd - k0, a.k_chunk)));
   const int nvalid = static_cast<int>(std::min<int64_t>(CB, a.Nd - n0));
-
-  for (int m = 0; m < MT; ++m)
-    for (int kk = threadIdx.x; kk < a.k_chunk; kk += blockDim.x) {
-      const float v = (m < a.M && kk < kc) ? load_v(a, m, k0 + kk) : 0.f;
-      sv2[kk * MT + m] = make_float2(v, v);
-    }
-  for (int i = threadIdx.x; i < MT * CB; i += blockDim.x) part[i] = 0.f;
-  __syncthreads();
 
   // This warp's rows: k0 + warp + 8j.  Their shift s is the same for all j.
   const int nrows = (kc > warp) ? (kc - warp + kRes - 1) / kRes : 0;
@@ -147,25 +140,34 @@ __global__ void __launch_bounds__(kFmaWarps * 32, 2) skinny_fma_kernel(SkinnyArg
   const bool all_fast = win0 >= a.w_lo &&
                         win0 + static_cast<uintptr_t>(nrows > 0 ? nrows - 1 : 0) * step + 512 <= a.w_hi;
 
+  auto load_row = [&](int j) -> uint4 {
+    const uintptr_t c = win0 + static_cast<uintptr_t>(j) * step + 16u * lane;
+    if (!need || j >= nrows) return make_uint4(0u, 0u, 0u, 0u);
+    return all_fast ? ld_nc_v4(c) : chunk16(c, a.w_lo, a.w_hi);
+  };
+
+  // Rolling pipeline: U rows in flight; consuming row j issues row j + U
+  // into the same register slot.  The first U rows of W do not depend on V,
+  // so they are in flight before waiting for the launch that writes V.
+  uint4 cur[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) cur[u] = load_row(u);
+  if (a.after_previous) griddep_wait();
+
+  for (int m = 0; m < MT; ++m)
+    for (int kk = threadIdx.x; kk < a.k_chunk; kk += blockDim.x) {
+      const float v = (m < a.M && kk < kc) ? load_v(a, m, k0 + kk) : 0.f;
+      sv2[kk * MT + m] = make_float2(v, v);
+    }
+  for (int i = threadIdx.x; i < MT * CB; i += blockDim.x) part[i] = 0.f;
+  __syncthreads();
+
   float2 acc[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[m][i] = make_float2(0.f, 0.f);
 
-  auto load_row = [&](int j) -> uint4 {
-    const uintptr_t win = win0 + static_cast<uintptr_t>(j) * step;
-    if (!need || j >= nrows) return make_uint4(0u, 0u, 0u, 0u);
-    if (all_fast) return ld_nc_v4(win + 16u * lane);
-    const bool fast = win >= a.w_lo && win + 512 <= a.w_hi;
-    return window_chunk(win + 16u * lane, true, fast, a.w_lo, a.w_hi);
-  };
-
-  // Rolling pipeline: U rows in flight; consuming row j issues row j + U
-  // into the same register slot.
-  uint4 cur[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) cur[u] = load_row(u);
   for (int j0 = 0; j0 < nrows; j0 += U) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -283,6 +285,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
   constexpr int CB = kMmaCB;
   extern __shared__ __align__(16) float smem[];
   uint4* sfrag = reinterpret_cast<uint4*>(smem);                      // [k_chunk/128][8][32][2]
+  griddep_launch_dependents();
   float* part = smem + a.k_chunk * 16;                                // [16][CB]
   uint8_t* bufs = reinterpret_cast<uint8_t*>(part + 16 * CB);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -292,6 +295,34 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
   const int64_t k0 = static_cast<int64_t>(blockIdx.y) * a.k_chunk;
   const int kc = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(a.Kd - k0, a.k_chunk)));
   const int nvalid = static_cast<int>(std::min<int64_t>(CB, a.Nd - n0));
+
+  MmaWarp w;
+  const uintptr_t row0 = reinterpret_cast<uintptr_t>(a.W + (k0 + res) * a.ldw + n0);
+  const int s = static_cast<int>((row0 >> 1) & 7u);
+  w.win0 = row0 & ~static_cast<uintptr_t>(15);
+  w.step = static_cast<uintptr_t>(kRes * a.ldw * 2);
+  w.lo = a.w_lo;
+  w.hi = a.w_hi;
+  w.nrows = (kc > res) ? (kc - res + kRes - 1) / kRes : 0;
+  w.lane = lane;
+  w.chunk = 8 * half + (lane & 7);
+  const int c0 = 8 * w.chunk - s;  // first column of the lane's load chunk
+  w.need = (c0 < nvalid) && (c0 + 8 > 0);
+  const int nsteps = (w.nrows + 15) / 16;
+
+  float d[8][4];
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[t][i] = 0.f;
+
+  // The first k-steps' rows of W do not depend on V: issue them before
+  // waiting for the launch that writes V.
+  uint4 c_a[4], c_b[4], c_c[4];
+  mma_issue(w, 0, c_a);
+  mma_issue(w, 1, c_b);
+  mma_issue(w, 2, c_c);
+  if (a.after_previous) griddep_wait();
 
   // Fragment element e of lane f (g = f/4, tq = f%4) for residue res and
   // k-step j: token g or g+8, local row res + 8·(16j + i) with
@@ -326,30 +357,6 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
   for (int i = threadIdx.x; i < 16 * CB; i += blockDim.x) part[i] = 0.f;
   __syncthreads();
 
-  MmaWarp w;
-  const uintptr_t row0 = reinterpret_cast<uintptr_t>(a.W + (k0 + res) * a.ldw + n0);
-  const int s = static_cast<int>((row0 >> 1) & 7u);
-  w.win0 = row0 & ~static_cast<uintptr_t>(15);
-  w.step = static_cast<uintptr_t>(kRes * a.ldw * 2);
-  w.lo = a.w_lo;
-  w.hi = a.w_hi;
-  w.nrows = (kc > res) ? (kc - res + kRes - 1) / kRes : 0;
-  w.lane = lane;
-  w.chunk = 8 * half + (lane & 7);
-  const int c0 = 8 * w.chunk - s;  // first column of the lane's load chunk
-  w.need = (c0 < nvalid) && (c0 + 8 > 0);
-  const int nsteps = (w.nrows + 15) / 16;
-
-  float d[8][4];
-#pragma unroll
-  for (int t = 0; t < 8; ++t)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[t][i] = 0.f;
-
-  uint4 c_a[4], c_b[4], c_c[4];
-  mma_issue(w, 0, c_a);
-  mma_issue(w, 1, c_b);
-  mma_issue(w, 2, c_c);
   for (int j = 0; j < nsteps; j += kMmaInflight) {
     mma_consume<V_F32>(w, j, c_a, tbuf, sfrag, res, d);
     mma_issue(w, j + 3, c_a);
@@ -406,7 +413,7 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms) {
   // partial-sum atomics.
   // Fixed cost of a CTA (staging V, zeroing, the atomics and the last-CTA
   // write), in rows of W.
-  const int64_t overhead = (p.kind == SkinnyKind::kFma) ? 48 : 192;
+  const int64_t overhead = (p.kind == SkinnyKind::kFma) ? 160 : 256;
   const int64_t max_splits = std::max<int64_t>(1, std::min<int64_t>(512, (Kd + gran - 1) / gran));
   double best = 1e300;
   p.k_chunk = static_cast<int>(cap);
@@ -437,19 +444,28 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms) {
   return p;
 }
 
-cudaError_t launch_skinny(const SkinnyPlan& p, const SkinnyArgs& args, cudaStream_t stream) {
-  dim3 grid(p.col_blocks, p.splits);
-  dim3 block(p.threads);
+cudaError_t launch_skinny(const SkinnyPlan& p, const SkinnyArgs& args, cudaStream_t stream,
+                          bool dependent) {
   SkinnyArgs a = args;
   a.k_chunk = p.k_chunk;
   a.splits = p.splits;
+  a.after_previous = dependent ? 1 : 0;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.col_blocks, p.splits);
+  cfg.blockDim = dim3(p.threads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
   cudaError_t e = cudaSuccess;
   auto go = [&](auto kern) {
     // Allow the largest dynamic shared memory any plan asks for.
     e = ensure_max_smem(reinterpret_cast<const void*>(kern), kSkinnyMaxSmem);
     if (e != cudaSuccess) return;
-    kern<<<grid, block, p.smem, stream>>>(a);
-    e = cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, kern, a);
   };
   if (p.kind == SkinnyKind::kFma) {
     if (p.mt == 1) go(skinny_fma_kernel<1>);

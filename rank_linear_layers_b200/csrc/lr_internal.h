@@ -48,6 +48,7 @@ struct SkinnyArgs {
   int64_t ld_out;
   const __nv_bfloat16* bias;
   WaitCtl wait;             // bounded waits on the copy pipeline
+  int after_previous;       // V is written by the previous launch (PDL wait)
 };
 
 enum class SkinnyKind { kFma, kMma };
@@ -64,7 +65,11 @@ struct SkinnyPlan {
 };
 
 SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms);
-cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& args, cudaStream_t stream);
+// With `dependent`, the launch may start while the previous launch on the
+// stream still runs (programmatic dependent launch); the kernel loads its
+// first rows of W and then waits for that launch before reading V.
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& args, cudaStream_t stream,
+                          bool dependent = false);
 
 // ------------------------------------------------------------------ prefill
 // C[Mr, Nc] = Aop[Mr, Kc] · Bop[Kc, Nc] (+ bias), bf16 in, fp32 accumulate,
@@ -94,6 +99,11 @@ constexpr int kGemmStages = 4;
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm(const GemmArgs& args, const GemmMaps& maps, int num_sms,
                         cudaStream_t stream);
+// The same on CTA pairs (2-SM MMA, 256×256 tiles).  The A map's box must be
+// {64, 128} and the B map's {64, 64}, as for launch_gemm.
+size_t gemm_pair_smem_bytes();
+cudaError_t launch_gemm_pair(const GemmArgs& args, const GemmMaps& maps, int num_sms,
+                             cudaStream_t stream);
 
 // Copy a [rows, cols] bf16 matrix with any 2-byte-aligned base and pitch lds
 // into dst (16-byte-aligned base, pitch ldd >= cols rounded up to 8).

@@ -37,9 +37,9 @@ __device__ __forceinline__ uint32_t ld_u16_or0(uintptr_t p, uintptr_t lo, uintpt
   return h;
 }
 
-// The aligned 16-byte chunk at a, with bytes outside [lo, hi) read as zero.
-__device__ __forceinline__ uint4 chunk16(uintptr_t a, uintptr_t lo, uintptr_t hi) {
-  if (a >= lo && a + 16 <= hi) return ld_nc_v4(a);
+// A chunk that straddles the tensor's first or last byte: element by element
+// (rare; kept out of line so that unrolled loops stay small).
+static __device__ __noinline__ uint4 chunk16_edge(uintptr_t a, uintptr_t lo, uintptr_t hi) {
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (a + 16 <= lo || a >= hi) return v;
   v.x = ld_u16_or0(a + 0, lo, hi) | (ld_u16_or0(a + 2, lo, hi) << 16);
@@ -47,6 +47,12 @@ __device__ __forceinline__ uint4 chunk16(uintptr_t a, uintptr_t lo, uintptr_t hi
   v.z = ld_u16_or0(a + 8, lo, hi) | (ld_u16_or0(a + 10, lo, hi) << 16);
   v.w = ld_u16_or0(a + 12, lo, hi) | (ld_u16_or0(a + 14, lo, hi) << 16);
   return v;
+}
+
+// The aligned 16-byte chunk at a, with bytes outside [lo, hi) read as zero.
+__device__ __forceinline__ uint4 chunk16(uintptr_t a, uintptr_t lo, uintptr_t hi) {
+  if (a >= lo && a + 16 <= hi) return ld_nc_v4(a);
+  return chunk16_edge(a, lo, hi);
 }
 
 __device__ __forceinline__ uint2 chunk8(uintptr_t a, uintptr_t lo, uintptr_t hi) {

@@ -19,40 +19,52 @@ namespace lr {
 namespace {
 
 constexpr int kRepackWarps = 8;
-constexpr int kRepackU = 4;  // row segments in flight per warp
+constexpr int kRepackU = 8;  // row segments in flight per warp
+constexpr int kRepackCtasPerSm = 2;
 
-// Task t = (row, 256-column segment).  Each warp takes kRepackU tasks at a
-// time (grid-stride), loads them all, then realigns and stores them.
+// The matrix is cut into 256-column segments of each row.  The grid's warps
+// are split into `segs` equal groups; the warps of group j copy segment j of
+// rows g, g + G, g + 2G, ... (G warps per group, g the warp's index in it),
+// through a rolling pipeline of kRepackU register slots: finishing row i
+// issues row i + kRepackU in its slot.  Only the start needs a division.
 __global__ void __launch_bounds__(kRepackWarps * 32) repack_rows_kernel(
     const __nv_bfloat16* __restrict__ src, int64_t lds, uintptr_t lo, uintptr_t hi,
     __nv_bfloat16* __restrict__ dst, int64_t ldd, int64_t rows, int64_t cols) {
   const int lane = threadIdx.x & 31;
-  const int64_t segs = (cols + 255) / 256;
-  const int64_t tasks = rows * segs;
-  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t t0 = warp_global * kRepackU; t0 < tasks; t0 += nwarps * kRepackU) {
-    uint4 cur[kRepackU], ext[kRepackU];
+  const int segs = static_cast<int>((cols + 255) / 256);
+  const int w = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int W = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
+  const int G = W / segs;  // warps per segment (the launch makes it >= 1)
+  if (w >= G * segs) return;
+  const int seg = w % segs, g = w / segs;
+  const int64_t c0 = static_cast<int64_t>(seg) * 256;
+  const int nv = static_cast<int>(std::min<int64_t>(256, cols - c0));
+  const int64_t mine = (rows > g) ? (rows - g + G - 1) / G : 0;  // rows of this warp
+  const __nv_bfloat16* s0 = src + static_cast<int64_t>(g) * lds + c0;
+  const int64_t sstep = static_cast<int64_t>(G) * lds;
+  __nv_bfloat16* d0 = dst + static_cast<int64_t>(g) * ldd + c0;
+  const int64_t dstep = static_cast<int64_t>(G) * ldd;
+
+  uint4 cur[kRepackU], ext[kRepackU];
+#pragma unroll
+  for (int u = 0; u < kRepackU; ++u)
+    seg16_issue(s0 + u * sstep, lane, 32, u < mine ? nv : 0, lo, hi, cur[u], ext[u]);
+  for (int64_t i0 = 0; i0 < mine; i0 += kRepackU) {
 #pragma unroll
     for (int u = 0; u < kRepackU; ++u) {
-      const int64_t t = t0 + u;
-      const int64_t row = t / segs, c0 = (t % segs) * 256;
-      const int nv = (t < tasks) ? static_cast<int>(std::min<int64_t>(256, cols - c0)) : 0;
-      seg16_issue(src + row * lds + c0, lane, 32, nv, lo, hi, cur[u], ext[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kRepackU; ++u) {
-      const int64_t t = t0 + u;
-      if (t >= tasks) break;
-      const int64_t row = t / segs, c0 = (t % segs) * 256;
-      const int nv = static_cast<int>(std::min<int64_t>(256, cols - c0));
-      const uint4 v = seg16_finish(cur[u], ext[u], seg_shift(src + row * lds + c0), lane, 32, nv);
+      const int64_t i = i0 + u;
+      if (i >= mine) break;
+      const __nv_bfloat16* sp = s0 + i * sstep;
+      const uint4 v = seg16_finish(cur[u], ext[u], seg_shift(sp), lane, 32, nv);
+      // Refill the slot with row i + U before storing this one.
+      seg16_issue(sp + kRepackU * sstep, lane, 32, i + kRepackU < mine ? nv : 0, lo, hi, cur[u],
+                  ext[u]);
       const int c = 8 * lane;
       if (c < nv) {
         // dst rows are 16-byte aligned and c0 + c is a multiple of 8: the
         // chunk is aligned; elements past nv are zero, and the pitch covers
         // them (ldd >= cols rounded up to 8).
-        *reinterpret_cast<uint4*>(dst + row * ldd + c0 + c) = v;
+        *reinterpret_cast<uint4*>(d0 + i * dstep + c) = v;
       }
     }
   }
@@ -65,10 +77,11 @@ cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_byte
                           int num_sms, cudaStream_t stream) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   const uintptr_t lo = reinterpret_cast<uintptr_t>(src);
-  const int64_t tasks = rows * ((cols + 255) / 256);
-  const int64_t warps_needed = (tasks + kRepackU - 1) / kRepackU;
-  const int64_t blocks_needed = (warps_needed + kRepackWarps - 1) / kRepackWarps;
-  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks_needed, num_sms * 8)));
+  // Enough warps that every segment gets at least one and the SMs fill.
+  const int64_t segs = (cols + 255) / 256;
+  const int64_t warps_wanted = std::max<int64_t>(segs, std::min<int64_t>(
+      segs * rows, static_cast<int64_t>(num_sms) * kRepackCtasPerSm * kRepackWarps));
+  const int blocks = static_cast<int>(std::max<int64_t>(1, (warps_wanted + kRepackWarps - 1) / kRepackWarps));
   repack_rows_kernel<<<blocks, kRepackWarps * 32, 0, stream>>>(src, lds, lo, lo + src_bytes, dst,
                                                                ldd, rows, cols);
   return cudaGetLastError();

@@ -192,7 +192,7 @@ extern "C" lr_status lr_linear_decode_static(const void* X, const void* A, const
   a.out_bf16 = static_cast<__nv_bfloat16*>(Y);
   a.ld_out = N;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
-  e = launch_skinny(p2, a, stream);
+  e = launch_skinny(p2, a, stream, true);
   if (e != cudaSuccess) return fail(e);
   note_launches(1);
   return LR_OK;

@@ -259,6 +259,199 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The same GEMM on pairs of SMs (a cluster of two CTAs, tcgen05 cta_group::2):
+// a pair computes a 256×256 tile; CTA r of the pair loads rows
+// [128r, 128r+128) of the A tile and columns [128r, 128r+128) of the B tile,
+// and its TMEM receives rows [128r, 128r+128) × all 256 columns of the
+// result.  Per SM a k block moves 32 KB (16 KB of A, 16 KB of B) instead of
+// 48 KB for the same tensor-core time, so shared-memory traffic drops by a
+// third and six stages fit.  The even CTA issues the MMAs; its commits
+// arrive on the barriers of both CTAs; the odd CTA's TMA loads complete on
+// the even CTA's full barrier; both epilogues release the accumulator on the
+// even CTA's barrier.
+constexpr int P_BM = 256;           // pair tile rows (128 per CTA)
+constexpr int P_BN = 256;           // pair tile columns (128 loaded per CTA)
+constexpr int P_STAGES = 6;
+constexpr int P_A_STAGE = 128 * BK * 2;  // 16 KB
+constexpr int P_B_STAGE = 128 * BK * 2;  // 16 KB (this CTA's half of B)
+constexpr int P_STAGE = P_A_STAGE + P_B_STAGE;
+constexpr int P_EPI_ARRIVALS = 2 * EPI_WARPS;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
+                          const __grid_constant__ CUtensorMap map_b, const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + P_STAGES * P_STAGE);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* fin = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1u);   // the even CTA's expect_tx; both CTAs' bytes
+      mbar_init(&empty[s], 1u);  // one multicast commit per stage
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1u);
+      mbar_init(&tempty[i], P_EPI_ARRIVALS);
+    }
+    mbar_init(fin, 1u);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == TMA_WARP && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int tiles_m = (g.Mr + P_BM - 1) / P_BM;
+  const int tiles_n = (g.Nc + P_BN - 1) / P_BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+  const int num_kb = (g.Kc + BK - 1) / BK;
+  int issued_phase[P_STAGES];
+#pragma unroll
+  for (int s = 0; s < P_STAGES; ++s) issued_phase[s] = -1;
+  bool ok = true;
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int tile = cluster; tile < num_tiles && ok; tile += clusters) {
+        const int m_blk = tile % tiles_m, n_blk = tile / tiles_m;
+        const int row0 = m_blk * P_BM + static_cast<int>(rank) * 128;
+        const int col0 = n_blk * P_BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereProducer)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
+          uint8_t* a_dst = base + s * P_STAGE;
+          uint8_t* b_dst = a_dst + P_A_STAGE;
+          tma_load_2d_pair(a_dst, &map_a, &full[s], kb * BK, row0);
+          tma_load_2d_pair(b_dst, &map_b, &full[s], col0, kb * BK);
+          tma_load_2d_pair(b_dst + B_ATOM, &map_b, &full[s], col0 + 64, kb * BK);
+          issued_phase[s] = static_cast<int>(ph);
+          if (++s == P_STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (leader) {
+      const uint32_t idesc = idesc_bf16_f32(P_BM, P_BN, false, true);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int tile = cluster; tile < num_tiles && ok; tile += clusters, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait, kWhereMmaAcc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[s], ph, g.wait, kWhereMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const int krem = g.Kc - kb * BK;
+            const int nk = krem >= BK ? BK / 16 : (krem + 15) / 16;
+            const uint32_t a0 = smem_u32(base + s * P_STAGE);
+            const uint32_t b0 = a0 + P_A_STAGE;
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(b0 + kk * 2048, B_ATOM, 1024);
+              umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&empty[s], 0x3);
+          }
+          __syncwarp();
+          if (++s == P_STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair(&tfull[acc], 0x3);
+        __syncwarp();
+      }
+    }
+  } else if (warp < EPI_WARPS) {
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(g.c) & 15u) == 0) && ((g.ldc & 7) == 0);
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int it = 0;
+    for (int tile = cluster; tile < num_tiles && ok; tile += clusters, ++it) {
+      const int m_blk = tile % tiles_m, n_blk = tile / tiles_m;
+      const int acc = it & 1;
+      const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
+      if (!mbar_wait(&tfull[acc], aph, g.wait, kWhereEpilogue)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = m_blk * P_BM + static_cast<int>(rank) * 128 + warp * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < P_BN / 32; ++c) {
+        const int col0 = n_blk * P_BN + c * 32;
+        if (col0 >= g.Nc) break;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
+        tmem_ld_wait();
+        store_chunk(g, row, col0, v, vec_ok);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(acc * 8));
+    }
+  }
+
+  // Teardown.  Every wait above is bounded, so every thread gets here.
+  if (leader && warp == MMA_WARP && lane == 0) {
+    umma_commit_pair(fin, 0x1);
+    mbar_wait_drain(fin, 0u, 2000000000ull);
+  }
+  if (leader && warp == TMA_WARP && lane == 0 && !ok) {
+    // After a timeout: the pair's TMA loads complete on these barriers.
+    for (int s = 0; s < P_STAGES; ++s)
+      if (issued_phase[s] >= 0)
+        mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_phase[s]), 1000000ull);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 __global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
                                  const __nv_bfloat16* bias) {
   const int64_t total = M * N;
@@ -273,6 +466,23 @@ __global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64
 
 size_t gemm_smem_bytes() {
   return 1024 + static_cast<size_t>(STAGES) * STAGE + (2 * STAGES + 5) * sizeof(uint64_t) + 16;
+}
+
+size_t gemm_pair_smem_bytes() {
+  return 1024 + static_cast<size_t>(P_STAGES) * P_STAGE + (2 * P_STAGES + 5) * sizeof(uint64_t) +
+         16;
+}
+
+cudaError_t launch_gemm_pair(const GemmArgs& g, const GemmMaps& maps, int num_sms,
+                             cudaStream_t stream) {
+  const size_t smem = gemm_pair_smem_bytes();
+  cudaError_t e = ensure_max_smem(reinterpret_cast<const void*>(umma_gemm_pair_kernel),
+                                  static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int tiles = ((g.Mr + P_BM - 1) / P_BM) * ((g.Nc + P_BN - 1) / P_BN);
+  const int clusters = std::max(1, std::min(tiles, num_sms / 2));
+  umma_gemm_pair_kernel<<<2 * clusters, kGemmThreads, smem, stream>>>(maps.a, maps.b, g);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,

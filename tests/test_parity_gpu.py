@@ -86,6 +86,22 @@ def test_prefill_ragged(lr, M, K, r, N):
     compare(run_gpu(lr, p, lr.PATH_PREFILL), ref(p), f"prefill {M}x{K}x{r}x{N}")
 
 
+@pytest.mark.parametrize("M,K,r,N", [
+    (256, 512, 256, 512),      # one pair tile
+    (300, 333, 257, 517),      # ragged everywhere, odd K and r
+    (640, 1024, 1741, 700),
+    (2048, 4096, 1741, 4096),  # the prefill q_proj shape (sampled rows)
+])
+def test_pair_and_single_sm_kernels_agree(lr, M, K, r, N):
+    p = lrgen.lowrank_problem(M, K, r, N, seed=M + r, bias=True)
+    Yp = run_gpu(lr, p, lr.PATH_PREFILL_PAIR)
+    Y1 = run_gpu(lr, p, lr.PATH_PREFILL_1SM)
+    rows = np.arange(M) if M <= 640 else np.random.default_rng(1).choice(M, 64, replace=False)
+    Yr = ref(p, rows=rows)
+    compare(Yp[rows], Yr, "pair kernel")
+    compare(Y1[rows], Yr, "single-SM kernel")
+
+
 def test_decode_and_prefill_agree_at_m16(lr):
     p = lrgen.lowrank_problem(16, 512, 300, 640, seed=3, bias=True)
     Yd = run_gpu(lr, p, lr.PATH_DECODE)
