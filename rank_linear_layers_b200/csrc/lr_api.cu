@@ -277,7 +277,7 @@ bool tma_ok(const void* p, int64_t ld) {
 // One prefill GEMM: C = a · b (+bias), both operands already TMA-able.
 lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, const void* b,
                int64_t ldb, void* c, int64_t ldc, const void* bias, int64_t Mr, int64_t Nc,
-               int64_t Kc) {
+               int64_t Kc, bool pdl = false, bool dep_a = false, bool dep_b = false) {
   GemmArgs g{};
   g.Mr = static_cast<int>(Mr);
   g.Nc = static_cast<int>(Nc);
@@ -288,6 +288,9 @@ lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, c
   g.tiles_m = static_cast<int>((Mr + kGemmBM - 1) / kGemmBM);
   g.tiles_n = static_cast<int>((Nc + kGemmBN - 1) / kGemmBN);
   g.wait = wait_ctl(d);
+  g.pdl = pdl ? 1 : 0;
+  g.dep_a = dep_a ? 1 : 0;
+  g.dep_b = dep_b ? 1 : 0;
   GemmMaps maps{};
   lr_status st = tensor_map(&maps.a, a, Kc, Mr, lda, kGemmBK, kGemmBM);
   if (st != LR_OK) return st;
@@ -344,9 +347,13 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x)) != LR_OK) return st;
   if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a)) != LR_OK) return st;
   if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b)) != LR_OK) return st;
-  st = gemm(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K);
+  // Kernels after the first of the call start early (programmatic dependent
+  // launch) and load only user inputs before waiting for their predecessor.
+  const bool x_rp = (x.p != X), a_rp = (a.p != A), b_rp = (b.p != B);
+  const bool g1_pdl = x_rp || a_rp || b_rp;
+  st = gemm(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K, g1_pdl, x_rp, a_rp);
   if (st != LR_OK) return st;
-  return gemm(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r);
+  return gemm(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r, true, true, b_rp);
 }
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,

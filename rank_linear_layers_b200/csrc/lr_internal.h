@@ -84,6 +84,11 @@ struct GemmArgs {
   const __nv_bfloat16* bias;
   int tiles_m, tiles_n;
   WaitCtl wait;
+  // Programmatic dependent launch: when `pdl`, the kernel may start while the
+  // previous launch on the stream runs; operands flagged dep_a / dep_b are
+  // written by earlier launches of the same call and are loaded only after
+  // griddepcontrol.wait, the others are loaded before it.
+  int pdl, dep_a, dep_b;
 };
 
 struct GemmMaps {

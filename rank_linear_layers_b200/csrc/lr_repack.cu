@@ -30,6 +30,7 @@ constexpr int kRepackCtasPerSm = 2;
 __global__ void __launch_bounds__(kRepackWarps * 32) repack_rows_kernel(
     const __nv_bfloat16* __restrict__ src, int64_t lds, uintptr_t lo, uintptr_t hi,
     __nv_bfloat16* __restrict__ dst, int64_t ldd, int64_t rows, int64_t cols) {
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int segs = static_cast<int>((cols + 255) / 256);
   const int w = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);

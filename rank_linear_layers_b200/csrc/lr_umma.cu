@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -146,20 +147,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == TMA_WARP) {
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
+      auto load_a = [&](int s, int kb, int m_blk) {
+        tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
+      };
+      auto load_b = [&](int s, int kb, int n_blk) {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+          tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
+      };
+      // Under programmatic dependent launch, fill the first stages with the
+      // operands the previous launch does not write, wait for it, then add
+      // the rest.  The first STAGES stages are free on entry.
+      int pre = 0;
+      if (g.pdl) {
+        const int tile = blockIdx.x;
+        if (tile < num_tiles) {
+          const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
+          pre = num_kb < STAGES ? num_kb : STAGES;
+          for (int kb = 0; kb < pre; ++kb) {
+            mbar_arrive_expect_tx(&full[kb], A_STAGE + B_STAGE);
+            if (!g.dep_a) load_a(kb, kb, m_blk);
+            if (!g.dep_b) load_b(kb, kb, n_blk);
+          }
+          griddep_wait();
+          for (int kb = 0; kb < pre; ++kb) {
+            if (g.dep_a) load_a(kb, kb, m_blk);
+            if (g.dep_b) load_b(kb, kb, n_blk);
+            issued_phase[kb] = 0;
+          }
+        } else {
+          griddep_wait();
+        }
+      }
+      int s = pre % STAGES;
+      uint32_t ph = (pre == STAGES) ? 1u : 0u;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = (tile == static_cast<int>(blockIdx.x)) ? pre : 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereProducer)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
-          tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
-#pragma unroll
-          for (int c = 0; c < BN / 64; ++c)
-            tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
+          load_a(s, kb, m_blk);
+          load_b(s, kb, n_blk);
           issued_phase[s] = static_cast<int>(ph);
           if (++s == STAGES) {
             s = 0;
@@ -492,9 +523,17 @@ cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,
       ensure_max_smem(reinterpret_cast<const void*>(umma_gemm_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = g.tiles_m * g.tiles_n;
-  const int grid = std::max(1, std::min(tiles, num_sms));
-  umma_gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(maps.a, maps.b, g);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(std::max(1, std::min(tiles, num_sms)));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel, maps.a, maps.b, g);
 }
 
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
