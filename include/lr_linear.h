@@ -170,6 +170,16 @@ int lr_last_cuda_error(void);
 lr_status lr_set_path(int path);
 lr_status lr_set_wait_limit_ns(int64_t ns);
 
+/*
+ * lr_set_withhold_first_stage — testing failure detection only.  With on = 1,
+ * the prefill kernels' copy thread never fills the first pipeline stage of
+ * its first tile, so the tensor-core thread's bounded wait on it runs out:
+ * the kernel records LR_ERR_TIMEOUT in the device status word, waits for its
+ * own copies and MMAs, frees its tensor memory and returns (Y is then not
+ * written).  Nothing faults or hangs.  on = 0 (the default) turns it off.
+ */
+lr_status lr_set_withhold_first_stage(int on);
+
 /* Counts the kernels launched by this library in this process. */
 int64_t lr_kernel_launch_count(void);
 

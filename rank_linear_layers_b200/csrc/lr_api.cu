@@ -22,6 +22,7 @@ thread_local int g_last_cuda_error = 0;
 std::atomic<int> g_path{0};
 std::atomic<long long> g_wait_ns{0};
 std::atomic<long long> g_launches{0};
+std::atomic<int> g_withhold{0};
 constexpr long long kDefaultWaitNs = 2000000000LL;
 
 struct DeviceInfo {
@@ -288,6 +289,7 @@ lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, c
   g.tiles_m = static_cast<int>((Mr + kGemmBM - 1) / kGemmBM);
   g.tiles_n = static_cast<int>((Nc + kGemmBN - 1) / kGemmBN);
   g.wait = wait_ctl(d);
+  g.withhold_first_stage = g_withhold.load();
   g.pdl = pdl ? 1 : 0;
   g.dep_a = dep_a ? 1 : 0;
   g.dep_b = dep_b ? 1 : 0;
@@ -589,6 +591,12 @@ lr_status lr_set_wait_limit_ns(int64_t ns) {
 }
 
 int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
+
+lr_status lr_set_withhold_first_stage(int on) {
+  if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
+  g_withhold.store(on);
+  return LR_OK;
+}
 
 lr_status lr_release_workspaces(void) {
   std::lock_guard<std::mutex> lk(g_mu);

@@ -89,6 +89,9 @@ struct GemmArgs {
   // written by earlier launches of the same call and are loaded only after
   // griddepcontrol.wait, the others are loaded before it.
   int pdl, dep_a, dep_b;
+  // Testing only: the producer withholds stage 0 of its first tile, so the
+  // MMA's bounded wait on it runs out (failure-detection test).
+  int withhold_first_stage;
 };
 
 struct GemmMaps {

@@ -164,13 +164,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (tile < num_tiles) {
           const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
           pre = num_kb < STAGES ? num_kb : STAGES;
-          for (int kb = 0; kb < pre; ++kb) {
+          const int first = g.withhold_first_stage ? 1 : 0;
+          for (int kb = first; kb < pre; ++kb) {
             mbar_arrive_expect_tx(&full[kb], A_STAGE + B_STAGE);
             if (!g.dep_a) load_a(kb, kb, m_blk);
             if (!g.dep_b) load_b(kb, kb, n_blk);
           }
           griddep_wait();
-          for (int kb = 0; kb < pre; ++kb) {
+          for (int kb = first; kb < pre; ++kb) {
             if (g.dep_a) load_a(kb, kb, m_blk);
             if (g.dep_b) load_b(kb, kb, n_blk);
             issued_phase[kb] = 0;
@@ -188,10 +189,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
-          load_a(s, kb, m_blk);
-          load_b(s, kb, n_blk);
-          issued_phase[s] = static_cast<int>(ph);
+          if (!(g.withhold_first_stage && kb == 0 && tile == static_cast<int>(blockIdx.x))) {
+            mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
+            load_a(s, kb, m_blk);
+            load_b(s, kb, n_blk);
+            issued_phase[s] = static_cast<int>(ph);
+          }
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
