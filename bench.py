@@ -281,6 +281,94 @@ def run_reference(args):
     return 0
 
 
+def _dev_bits(bits, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def sweep_times(lr, dev, l2, ranks, steps=20, warmup=3):
+    """Time per call at M = K = N = 4096 for each rank.  X ~ N(0,1),
+    A ~ N(0, 1/K), B ~ N(0, 1/1000): the A and B of each rank are the leading
+    columns / rows of one seeded draw (values do not affect the timing)."""
+    import torch
+    Mw, Kw, Nw = 4096, 4096, 4096
+    rmax = max(ranks)
+    X0 = _dev_bits(lrgen.normal_bf16(0, 1, (Mw, Kw)), dev)
+    Af = _dev_bits(lrgen.normal_bf16(0, 2, (Kw, rmax), 1.0 / math.sqrt(Kw)), dev)
+    Bf = _dev_bits(lrgen.normal_bf16(0, 3, (rmax, Nw), 1.0 / math.sqrt(1000)), dev)
+    Xs = [X0] + [X0.clone() for _ in range(max(1, math.ceil(2 * l2 / (X0.numel() * 2))))]
+    Y = torch.empty((Mw, Nw), dtype=torch.bfloat16, device=dev)
+    out = {}
+    for r in ranks:
+        A = Af[:, :r].contiguous()
+        B = Bf[:r].contiguous()
+
+        def st(i, A=A, B=B):
+            lr.lr_linear(Xs[i % len(Xs)], A, B, None, Y=Y)
+        tt = time_steps(st, steps, warmup) / steps
+        out[r] = {"us": tt * 1e6, "ps_per_flop": tt / acc.flops(Mw, Kw, r, Nw) * 1e12}
+    return out
+
+
+def misalignment_check(lr, dev, l2, ranks=range(1000, 1009)):
+    """Misaligned ranks against the nearest multiple of 8 (both neighbours
+    at r = 4 mod 8), in time per FLOP."""
+    t = sweep_times(lr, dev, l2, list(ranks))
+    worst = 0.0
+    rows = {}
+    for r, v in t.items():
+        if r % 8 == 0:
+            continue
+        lo, hi = r - r % 8, r - r % 8 + 8
+        near = [lo] if r % 8 < 4 else ([hi] if r % 8 > 4 else [lo, hi])
+        near = [n for n in near if n in t]
+        if not near:
+            continue
+        dev_pct = max(v["ps_per_flop"] / t[n]["ps_per_flop"] - 1.0 for n in near)
+        rows[r] = round(dev_pct * 100, 2)
+        worst = max(worst, dev_pct)
+    return {"workload": "M=K=N=4096, r=1000..1008", "us": {r: round(v["us"], 2) for r, v in t.items()},
+            "pct_slower_than_nearest_aligned_per_flop": rows, "worst_pct": round(worst * 100, 2),
+            "target_pct": 5.0}
+
+
+def layer_bench(lr, dev, peaks, n_int=14336):
+    """A full factorised Llama-3-8B decoder layer through lr_linear_group."""
+    import torch
+    res = {}
+    for Ml in (1, 4096):
+        layer = lrgen.decoder_layer(Ml, seed=7, n_int=n_int)
+        xs = {k: _dev_bits(v, dev) for k, v in layer["inputs"].items()}
+        P = layer["projs"]
+        packed = torch.empty((Ml, 2 * n_int), dtype=torch.bfloat16, device=dev)
+        entries, keep = [], []
+        for name, p in P.items():
+            A, B = _dev_bits(p["A"], dev), _dev_bits(p["B"], dev)
+            keep += [A, B]
+            e = dict(X=xs[p["x"]], A=A, B=B, K=p["K"], r=p["r"], N=p["N"])
+            if name in ("gate", "up"):
+                e["Y_ptr"] = packed.data_ptr() + (0 if name == "gate" else 2 * n_int)
+                e["ld_y"] = 2 * n_int
+            else:
+                Yp = torch.empty((Ml, p["N"]), dtype=torch.bfloat16, device=dev)
+                keep.append(Yp)
+                e["Y"] = Yp
+            entries.append(e)
+        tl = time_steps(lambda i: lr.lr_linear_group(entries, Ml), 20, 3) / 20
+        projs = [dict(K=p["K"], r=p["r"], N=p["N"], x=p["x"]) for p in P.values()]
+        fl, by = acc.group_work(Ml, projs)
+        dense_by = sum(acc.dense_bytes(Ml, p["K"], p["N"]) for p in P.values())
+        dense_fl = sum(acc.dense_flops(Ml, p["K"], p["N"]) for p in P.values())
+        roof = acc.roofline(fl, by, peaks["bf16_tflops"], peaks["hbm_gbs"])
+        droof = acc.roofline(dense_fl, dense_by, peaks["bf16_tflops"], peaks["hbm_gbs"])
+        res[f"M{Ml}"] = {"us": tl * 1e6, "TFLOP/s": fl / tl / 1e12, "GB/s": by / tl / 1e9,
+                         "roofline_us": roof.t_roof_s * 1e6, "frac_roofline": roof.t_roof_s / tl,
+                         "dense_roofline_us": droof.t_roof_s * 1e6,
+                         "ranks": layer["ranks"], "keep_ratio": acc.keep_ratio(
+                             [(p["K"], p["N"], p["r"]) for p in P.values()])}
+    return res
+
+
 def metric_name():
     return "low-rank linear TFLOP/s (prefill) and GB/s (decode) as % of B200 roofline"
 
@@ -413,6 +501,25 @@ def run_ours(args):
                     "dense_equiv_us_at_peak": acc.dense_bytes(dm, dk, dn) / (peaks["hbm_gbs"] * 1e9) * 1e6}
                 del Ads, Bds
 
+    # Dense X·W at the same M, K, N through the same kernels: is the
+    # factorised layer (15% fewer parameters) still slower?
+    dense = None
+    if not args.no_extra:
+        gen = torch.Generator(device=dev).manual_seed(0)
+        Wd = [(torch.randn((K, N), generator=gen, device=dev) / math.sqrt(K)).to(torch.bfloat16)
+              for _ in range(copies)]
+        Yd = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def dstep(i):
+            lr.lr_dense(Xs[i % copies], Wd[i % copies], None, Y=Yd)
+        tdd = time_steps(dstep, args.steps, args.warmup) / args.steps
+        dense = {"us": tdd * 1e6, "TFLOP/s": acc.dense_flops(M, K, N) / tdd / 1e12,
+                 "lowrank_over_dense_time": (t / args.steps) / tdd,
+                 "note": "lr_dense, same tcgen05 kernel, W [4096,4096] N(0,1/K)"}
+        del Wd
+    misalign = misalignment_check(lr, dev, l2) if not args.no_extra else None
+    layer = layer_bench(lr, dev, peaks) if not args.no_extra else None
+
     cb = cpu_baseline(p) if (rank == 0 and world == 1) else None
     if rank == 0:
         line = {
@@ -421,7 +528,8 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config_dict(), "roofline": roofline,
             "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches_timed),
-            "clocks": clk, "parity": parity, "decode": decode,
+            "clocks": clk, "parity": parity, "decode": decode, "dense": dense,
+            "misalignment": misalign, "layer": layer,
         }
         print(json.dumps(line))
     if world > 1:
@@ -438,6 +546,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the dense, misalignment and decoder-layer measurements")
+    ap.add_argument("--sweep", action="store_true",
+                    help="only the misalignment sweep r = 1000..1100 and {64,128,512,2048}")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed prefill steps (for ncu captures); numbers are not a bench line")
     args = ap.parse_args()
@@ -445,7 +557,40 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep()
     return run_ours(args)
+
+
+def run_sweep():
+    """The full misalignment sweep (M = K = N = 4096), one JSON line."""
+    import torch
+    import rank_linear_layers_b200 as lr
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ranks = list(range(1000, 1101)) + [64, 128, 512, 2048]
+    t = sweep_times(lr, dev, l2, ranks)
+    peaks = load_peaks()
+    rows = {}
+    worst = 0.0
+    for r in range(1000, 1101):
+        if r % 8 == 0:
+            continue
+        lo, hi = r - r % 8, r - r % 8 + 8
+        near = [n for n in ([lo] if r % 8 < 4 else ([hi] if r % 8 > 4 else [lo, hi])) if n in t]
+        d = max(t[r]["ps_per_flop"] / t[n]["ps_per_flop"] - 1.0 for n in near)
+        rows[r] = round(d * 100, 2)
+        worst = max(worst, d)
+    roof = {}
+    for r in ranks:
+        rf = acc.roofline(acc.flops(4096, 4096, r, 4096), acc.algorithmic_bytes(4096, 4096, r, 4096),
+                          peaks["bf16_tflops"], peaks["hbm_gbs"])
+        roof[r] = round(rf.t_roof_s / (t[r]["us"] * 1e-6), 3)
+    print(json.dumps({"sweep": "M=K=N=4096", "us": {r: round(v["us"], 2) for r, v in t.items()},
+                      "frac_roofline": roof, "pct_slower_than_nearest_aligned_per_flop": rows,
+                      "worst_pct": round(worst * 100, 2), "target_pct": 5.0}))
+    return 0
 
 
 if __name__ == "__main__":
