@@ -162,13 +162,20 @@ int lr_last_cuda_error(void);
  *   0 = automatic (M <= 16 decode, else prefill), 1 = force decode (M <= 16
  *   only; larger M returns LR_ERR_INVALID_ARG), 2 = force prefill, 3 = force
  *   prefill on single-SM tiles (the default prefill kernel), 4 = force prefill
- *   on CTA pairs (2-SM MMA, 256×256 tiles; M <= 128 still uses single SMs).
+ *   on CTA pairs (2-SM MMA, 256×256 tiles, GEMM1 and GEMM2 as two launches;
+ *   M <= 128 still uses single SMs).
  * lr_set_wait_limit_ns — time limit of every device-side bounded wait
  *   (default 2e9 ns); 0 restores the default.
- * Both are process-wide and take effect on the next call.
+ * lr_set_tile_n — column width of the prefill kernel's single-SM tiles:
+ *   0 (the default) lets the library choose per GEMM (a schedule model picks
+ *   the width that spreads the launch's tiles most evenly over the SMs);
+ *   32..256 in steps of 32 forces that width for every GEMM (for tests and
+ *   tuning).  Other values return LR_ERR_INVALID_ARG.
+ * All three are process-wide and take effect on the next call.
  */
 lr_status lr_set_path(int path);
 lr_status lr_set_wait_limit_ns(int64_t ns);
+lr_status lr_set_tile_n(int bn);
 
 /*
  * lr_set_withhold_first_stage — testing failure detection only.  With on = 1,

@@ -1,6 +1,7 @@
 // lr_api.cu — the C ABI of include/lr_linear.h: argument validation, path
 // selection, workspaces, TMA descriptors and status reporting.  Every step
 // of the layer itself runs in the kernels of lr_decode.cu and lr_umma.cu.
+#include <algorithm>
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
@@ -23,6 +24,7 @@ std::atomic<int> g_path{0};
 std::atomic<long long> g_wait_ns{0};
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_withhold{0};
+std::atomic<int> g_tile_n{0};
 constexpr long long kDefaultWaitNs = 2000000000LL;
 
 struct DeviceInfo {
@@ -38,6 +40,11 @@ struct Workspace {
   char* ptr = nullptr;
   size_t cap = 0;
   size_t zero_bytes = 0;  // prefix that is all-zero between calls
+  // Row-block counters of the chain kernel: two banks of n_ctrs, used by
+  // alternate launches.
+  unsigned int* ctrs = nullptr;
+  size_t n_ctrs = 0;
+  unsigned int launches = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
@@ -53,9 +60,10 @@ struct MapKey {
   const void* ptr;
   uint64_t inner, outer, stride;
   uint32_t box_inner, box_outer;
+  int swizzle;
   bool operator<(const MapKey& o) const {
-    return std::tie(ptr, inner, outer, stride, box_inner, box_outer) <
-           std::tie(o.ptr, o.inner, o.outer, o.stride, o.box_inner, o.box_outer);
+    return std::tie(ptr, inner, outer, stride, box_inner, box_outer, swizzle) <
+           std::tie(o.ptr, o.inner, o.outer, o.stride, o.box_inner, o.box_outer, o.swizzle);
   }
 };
 std::map<MapKey, CUtensorMap> g_maps;
@@ -102,12 +110,14 @@ lr_status get_encoder() {
   return LR_OK;
 }
 
-// 2-D bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
+// 2-D bf16 tensor map (128-byte swizzle unless `swizzle64`), out-of-bounds
+// elements read as zero (loads) or are not written (stores).
 lr_status tensor_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
-                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer) {
+                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer,
+                     bool swizzle64 = false) {
   lr_status st = get_encoder();
   if (st != LR_OK) return st;
-  MapKey key{ptr, inner, outer, row_stride_elems, box_inner, box_outer};
+  MapKey key{ptr, inner, outer, row_stride_elems, box_inner, box_outer, swizzle64 ? 64 : 128};
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_maps.find(key);
@@ -122,7 +132,8 @@ lr_status tensor_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_last_cuda_error = static_cast<int>(r);
@@ -275,10 +286,236 @@ bool tma_ok(const void* p, int64_t ld) {
   return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && (ld % 8 == 0);
 }
 
-// One prefill GEMM: C = a · b (+bias), both operands already TMA-able.
-lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, const void* b,
-               int64_t ldb, void* c, int64_t ldc, const void* bias, int64_t Mr, int64_t Nc,
-               int64_t Kc, bool pdl = false, bool dep_a = false, bool dep_b = false) {
+// Counter banks for one chain launch on `stream`: the launch's bank (zero)
+// and the other one (which the launch zeroes for the next).
+lr_status chain_counters(cudaStream_t stream, size_t n, unsigned int** bank,
+                         unsigned int** next, int* per_bank) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  if (n > w.n_ctrs) {
+    if (w.ctrs) {
+      LR_CUDA(cudaStreamSynchronize(stream));
+      LR_CUDA(cudaFree(w.ctrs));
+      w.ctrs = nullptr;
+      w.n_ctrs = 0;
+    }
+    const size_t cap = align_up(std::max<size_t>(n, 1024), 1024);
+    LR_CUDA(cudaMalloc(&w.ctrs, 2 * cap * sizeof(unsigned int)));
+    LR_CUDA(cudaMemsetAsync(w.ctrs, 0, 2 * cap * sizeof(unsigned int), stream));
+    w.n_ctrs = cap;
+  }
+  const unsigned int b = (w.launches++) & 1u;
+  *bank = w.ctrs + b * w.n_ctrs;
+  *next = w.ctrs + (1u - b) * w.n_ctrs;
+  *per_bank = static_cast<int>(w.n_ctrs);
+  return LR_OK;
+}
+
+// One launch of the chain kernel under construction.
+struct ChainBuild {
+  ChainMaps maps{};
+  ChainArgs args{};
+  int n_maps = 0;
+};
+
+// Tensor map for operand a (K-major, box 64 × 128 rows) or operand b
+// (MN-major, box 64 columns × 64 rows) of the chain kernel.
+lr_status chain_map(ChainBuild& cb, const void* p, int64_t inner, int64_t outer, int64_t ld,
+                    bool operand_a, int* idx) {
+  if (cb.n_maps >= kChainMaxMaps) return LR_ERR_UNSUPPORTED;
+  lr_status st = tensor_map(&cb.maps.m[cb.n_maps], p, static_cast<uint64_t>(inner),
+                            static_cast<uint64_t>(outer), static_cast<uint64_t>(ld), 64,
+                            operand_a ? kGemmBM : kGemmBK);
+  if (st != LR_OK) return st;
+  *idx = cb.n_maps++;
+  return LR_OK;
+}
+
+lr_status chain_problem(ChainBuild& cb, int map_a, int a_col0, int map_b, int64_t Mr, int64_t Nc,
+                        int64_t Kc, void* c, int64_t ldc, const void* bias, int wait_group,
+                        int signal_group, bool dep_a, bool dep_b) {
+  if (cb.args.n_prob >= kChainMaxProbs) return LR_ERR_UNSUPPORTED;
+  // C through TMA stores when its base and pitch allow, else plain stores.
+  int map_c = -1;
+  if (tma_ok(c, ldc) && cb.n_maps < kChainMaxMaps) {
+    lr_status st = tensor_map(&cb.maps.m[cb.n_maps], c, static_cast<uint64_t>(Nc),
+                              static_cast<uint64_t>(Mr), static_cast<uint64_t>(ldc), 32, 32, true);
+    if (st != LR_OK) return st;
+    map_c = cb.n_maps++;
+  }
+  ChainProblem& P = cb.args.p[cb.args.n_prob++];
+  P = ChainProblem{};
+  P.map_c = map_c;
+  P.Mr = static_cast<int>(Mr);
+  P.Nc = static_cast<int>(Nc);
+  P.Kc = static_cast<int>(Kc);
+  P.map_a = map_a;
+  P.map_b = map_b;
+  P.a_col0 = a_col0;
+  P.c = static_cast<__nv_bfloat16*>(c);
+  P.ldc = ldc;
+  P.bias = static_cast<const __nv_bfloat16*>(bias);
+  P.wait_group = wait_group;
+  P.signal_group = signal_group;
+  P.dep_a = dep_a ? 1 : 0;
+  P.dep_b = dep_b ? 1 : 0;
+  return LR_OK;
+}
+
+// ---- tile-width planning
+// Estimated time of one 64-deep k block of a 128 × bn tile.  Measured on
+// B200 (dense 4096³ at each width): 0.38 µs at bn = 64 rising to 0.44 µs at
+// bn = 256 — the copy pipeline, not the tensor core, sets the pace, so
+// narrow tiles buy little time per tile.
+double kblock_us(int bn) { return 0.37 + 0.07 * bn / 256.0; }
+double epilogue_us(int bn) { return 0.6 + 1.0 * bn / 256.0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Simulate the static round-robin schedule of the chain kernel.
+double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
+  int64_t total = 0;
+  for (int i = 0; i < a.n_prob; ++i)
+    total += ceil_div(a.p[i].Mr, kGemmBM) * ceil_div(a.p[i].Nc, bn[i]);
+  const int64_t G = std::max<int64_t>(1, std::min<int64_t>(total, sms));
+  std::vector<double> t(static_cast<size_t>(G), 0.0);
+  std::map<int, std::vector<double>> ready;
+  int64_t idx = 0;
+  double tail = 0.0;
+  for (int i = 0; i < a.n_prob; ++i) {
+    const ChainProblem& P = a.p[i];
+    const int64_t tm = ceil_div(P.Mr, kGemmBM), tn = ceil_div(P.Nc, bn[i]);
+    const double dur = static_cast<double>(ceil_div(P.Kc, kGemmBK)) * kblock_us(bn[i]) + 0.15;
+    std::vector<double>* sig = nullptr;
+    const std::vector<double>* wait = nullptr;
+    if (P.signal_group >= 0) {
+      sig = &ready[P.signal_group];
+      sig->assign(static_cast<size_t>(tm), 0.0);
+    }
+    if (P.wait_group >= 0) {
+      auto it = ready.find(P.wait_group);
+      if (it != ready.end()) wait = &it->second;
+    }
+    for (int64_t l = 0; l < tm * tn; ++l, ++idx) {
+      double& tc = t[static_cast<size_t>(idx % G)];
+      const int64_t m = l / tn;
+      double start = tc;
+      if (wait && m < static_cast<int64_t>(wait->size())) start = std::max(start, (*wait)[m]);
+      tc = start + dur;
+      if (sig) (*sig)[m] = std::max((*sig)[m], tc + epilogue_us(bn[i]));
+    }
+    tail = epilogue_us(bn[i]);
+  }
+  return *std::max_element(t.begin(), t.end()) + tail;
+}
+
+std::mutex g_plan_mu;
+std::map<std::vector<int64_t>, std::vector<int>> g_plans;
+
+// Choose each problem's tile width.  Candidates are the multiples of 32 up
+// to min(256, N rounded up to 32); two problems are searched jointly, more
+// by coordinate descent from the widest tiles.
+std::vector<int> plan_chain(const ChainArgs& a, int sms) {
+  const int forced = g_tile_n.load();
+  std::vector<int64_t> key{sms, forced};
+  for (int i = 0; i < a.n_prob; ++i) {
+    const ChainProblem& P = a.p[i];
+    key.insert(key.end(), {P.Mr, P.Nc, P.Kc, P.wait_group, P.signal_group});
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    auto it = g_plans.find(key);
+    if (it != g_plans.end()) return it->second;
+  }
+  std::vector<int> bn(static_cast<size_t>(a.n_prob), 256);
+  if (forced > 0) {
+    std::fill(bn.begin(), bn.end(), forced);
+  } else {
+    std::vector<std::vector<int>> cand(static_cast<size_t>(a.n_prob));
+    for (int i = 0; i < a.n_prob; ++i) {
+      const int top = static_cast<int>(std::min<int64_t>(256, ceil_div(a.p[i].Nc, 32) * 32));
+      for (int b = top; b >= 32; b -= 32) cand[i].push_back(b);
+      bn[i] = top;
+    }
+    double best = simulate_chain(a, bn, sms);
+    if (a.n_prob == 2) {
+      for (int b0 : cand[0])
+        for (int b1 : cand[1]) {
+          std::vector<int> tryb{b0, b1};
+          const double t = simulate_chain(a, tryb, sms);
+          if (t < best * 0.999) {
+            best = t;
+            bn = tryb;
+          }
+        }
+    } else {
+      for (int pass = 0; pass < 2; ++pass)
+        for (int i = 0; i < a.n_prob; ++i)
+          for (int b : cand[i]) {
+            std::vector<int> tryb = bn;
+            tryb[i] = b;
+            const double t = simulate_chain(a, tryb, sms);
+            if (t < best * 0.999) {
+              best = t;
+              bn = tryb;
+            }
+          }
+    }
+  }
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  if (g_plans.size() > 4096) g_plans.clear();
+  g_plans.emplace(key, bn);
+  return bn;
+}
+
+// Plan, number the tiles and launch.  The launch may start while the
+// previous kernel on the stream still runs (programmatic dependent launch);
+// the problems' dep_a / dep_b say which operands that kernel may write.
+lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
+  ChainArgs& a = cb.args;
+  if (a.n_prob == 0) return LR_OK;
+  const std::vector<int> bn = plan_chain(a, d->sms);
+  int64_t total = 0;
+  int groups = 0, stride = 1;
+  for (int i = 0; i < a.n_prob; ++i) {
+    ChainProblem& P = a.p[i];
+    P.bn = bn[i];
+    P.tiles_m = static_cast<int>(ceil_div(P.Mr, kGemmBM));
+    P.tiles_n = static_cast<int>(ceil_div(P.Nc, P.bn));
+    P.tile_begin = static_cast<int>(total);
+    total += static_cast<int64_t>(P.tiles_m) * P.tiles_n;
+    if (total > kMaxDim) return LR_ERR_UNSUPPORTED;
+    if (P.signal_group >= 0) {
+      groups = std::max(groups, P.signal_group + 1);
+      stride = std::max(stride, P.tiles_m);
+    }
+  }
+  for (int i = 0; i < a.n_prob; ++i) {
+    ChainProblem& P = a.p[i];
+    if (P.wait_group < 0) continue;
+    P.wait_count = 0;
+    for (int j = 0; j < i; ++j)
+      if (a.p[j].signal_group == P.wait_group) P.wait_count += 4 * a.p[j].tiles_n;
+  }
+  a.total_tiles = static_cast<int>(total);
+  if (total == 0) return LR_OK;
+  a.ctr_stride = stride;
+  lr_status st = chain_counters(stream, static_cast<size_t>(std::max(groups, 1)) * stride,
+                                &a.counters, &a.counters_next, &a.n_counters);
+  if (st != LR_OK) return st;
+  a.wait = wait_ctl(d);
+  a.pdl = 1;
+  a.withhold_first_stage = g_withhold.load();
+  const int grid = static_cast<int>(std::min<int64_t>(total, d->sms));
+  return launched(launch_chain(cb.maps, a, grid, stream));
+}
+
+// One GEMM on CTA pairs (path 4): C = a · b (+bias).
+lr_status gemm_pair(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, const void* b,
+                    int64_t ldb, void* c, int64_t ldc, const void* bias, int64_t Mr, int64_t Nc,
+                    int64_t Kc) {
   GemmArgs g{};
   g.Mr = static_cast<int>(Mr);
   g.Nc = static_cast<int>(Nc);
@@ -286,22 +523,13 @@ lr_status gemm(DeviceInfo* d, cudaStream_t stream, const void* a, int64_t lda, c
   g.c = static_cast<__nv_bfloat16*>(c);
   g.ldc = ldc;
   g.bias = static_cast<const __nv_bfloat16*>(bias);
-  g.tiles_m = static_cast<int>((Mr + kGemmBM - 1) / kGemmBM);
-  g.tiles_n = static_cast<int>((Nc + kGemmBN - 1) / kGemmBN);
   g.wait = wait_ctl(d);
-  g.withhold_first_stage = g_withhold.load();
-  g.pdl = pdl ? 1 : 0;
-  g.dep_a = dep_a ? 1 : 0;
-  g.dep_b = dep_b ? 1 : 0;
   GemmMaps maps{};
   lr_status st = tensor_map(&maps.a, a, Kc, Mr, lda, kGemmBK, kGemmBM);
   if (st != LR_OK) return st;
   st = tensor_map(&maps.b, b, Nc, Kc, ldb, 64, kGemmBK);
   if (st != LR_OK) return st;
-  // Single-SM tiles by default; CTA pairs (2-SM MMA, 256-row tiles) when
-  // selected with lr_set_path(4) (measured no faster on the prefill shapes).
-  if (Mr > kGemmBM && g_path.load() == 4) return launched(launch_gemm_pair(g, maps, d->sms, stream));
-  return launched(launch_gemm(g, maps, d->sms, stream));
+  return launched(launch_gemm_pair(g, maps, d->sms, stream));
 }
 
 // A TMA-able view of a [rows, cols] operand: itself, or a realigned copy in
@@ -316,8 +544,10 @@ size_t repack_bytes(const void* p, int64_t ld, int64_t rows, int64_t cols) {
   return align_up(static_cast<size_t>(rows) * align_up(static_cast<size_t>(cols), 8) * 2, 256);
 }
 
+// `*repacks` counts the repack launches of the call so far: all but the first
+// may start early (programmatic dependent launch).
 lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t ld, int64_t rows,
-                      int64_t cols, char** scratch, Operand* out) {
+                      int64_t cols, char** scratch, Operand* out, int* repacks) {
   if (tma_ok(p, ld)) {
     *out = Operand{p, ld};
     return LR_OK;
@@ -327,8 +557,9 @@ lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t
   *scratch += repack_bytes(p, ld, rows, cols);
   lr_status st = launched(launch_repack(static_cast<const __nv_bfloat16*>(p), ld,
                                         span_bytes(rows, cols, ld), dst, ldd, rows, cols, d->sms,
-                                        stream));
+                                        stream, *repacks > 0));
   if (st != LR_OK) return st;
+  ++*repacks;
   *out = Operand{dst, ldd};
   return LR_OK;
 }
@@ -346,16 +577,34 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   void* T = scratch;
   scratch += tbytes;
   Operand x, a, b;
-  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b)) != LR_OK) return st;
-  // Kernels after the first of the call start early (programmatic dependent
-  // launch) and load only user inputs before waiting for their predecessor.
-  const bool x_rp = (x.p != X), a_rp = (a.p != A), b_rp = (b.p != B);
-  const bool g1_pdl = x_rp || a_rp || b_rp;
-  st = gemm(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K, g1_pdl, x_rp, a_rp);
+  int repacks = 0;
+  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x, &repacks)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a, &repacks)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b, &repacks)) != LR_OK) return st;
+  if (g_path.load() == 4) {
+    // CTA-pair tiles: the two GEMMs as two launches.
+    st = gemm_pair(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K);
+    if (st != LR_OK) return st;
+    return gemm_pair(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r);
+  }
+  // One launch: GEMM1 T = X·A signals counter group 0 per 128-row block;
+  // GEMM2 Y = T·B + bias waits on it row block by row block.  The launch
+  // may overlap the kernel before it: after this call's repacks only the
+  // repacked operands depend on that kernel; with no repack, it is the
+  // caller's previous kernel, which may have written any input.
+  const bool after_repack = repacks > 0;
+  auto dep = [&](const void* used, const void* given) { return !after_repack || used != given; };
+  ChainBuild cb;
+  int mx, ma, mt, mb;
+  if ((st = chain_map(cb, x.p, K, M, x.ld, true, &mx)) != LR_OK) return st;
+  if ((st = chain_map(cb, a.p, r, K, a.ld, false, &ma)) != LR_OK) return st;
+  if ((st = chain_map(cb, T, r, M, ldt, true, &mt)) != LR_OK) return st;
+  if ((st = chain_map(cb, b.p, N, r, b.ld, false, &mb)) != LR_OK) return st;
+  st = chain_problem(cb, mx, 0, ma, M, r, K, T, ldt, nullptr, -1, 0, dep(x.p, X), dep(a.p, A));
   if (st != LR_OK) return st;
-  return gemm(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r, true, true, b_rp);
+  st = chain_problem(cb, mt, 0, mb, M, N, r, Y, ldy, bias, 0, -1, false, dep(b.p, B));
+  if (st != LR_OK) return st;
+  return run_chain(d, stream, cb);
 }
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
@@ -540,9 +789,19 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
     st = workspace(stream, 0, need, &zero, &scratch);
     if (st != LR_OK) return st;
     Operand x, w;
-    if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x)) != LR_OK) return st;
-    if ((st = tma_operand(d, stream, W, N, K, N, &scratch, &w)) != LR_OK) return st;
-    return gemm(d, stream, x.p, x.ld, w.p, w.ld, Y, N, bias, M, N, K);
+    int repacks = 0;
+    if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x, &repacks)) != LR_OK) return st;
+    if ((st = tma_operand(d, stream, W, N, K, N, &scratch, &w, &repacks)) != LR_OK) return st;
+    if (path == 4) return gemm_pair(d, stream, x.p, x.ld, w.p, w.ld, Y, N, bias, M, N, K);
+    ChainBuild cb;
+    int mx, mw;
+    if ((st = chain_map(cb, x.p, K, M, x.ld, true, &mx)) != LR_OK) return st;
+    if ((st = chain_map(cb, w.p, N, K, w.ld, false, &mw)) != LR_OK) return st;
+    const bool after_repack = repacks > 0;
+    st = chain_problem(cb, mx, 0, mw, M, N, K, Y, N, bias, -1, -1, !after_repack || x.p != X,
+                       !after_repack || w.p != W);
+    if (st != LR_OK) return st;
+    return run_chain(d, stream, cb);
   }
 }
 
@@ -592,6 +851,12 @@ lr_status lr_set_wait_limit_ns(int64_t ns) {
 
 int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
 
+lr_status lr_set_tile_n(int bn) {
+  if (bn < 0 || bn > 256 || bn % 32 != 0) return LR_ERR_INVALID_ARG;
+  g_tile_n.store(bn);
+  return LR_OK;
+}
+
 lr_status lr_set_withhold_first_stage(int on) {
   if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
   g_withhold.store(on);
@@ -603,10 +868,11 @@ lr_status lr_release_workspaces(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_ws) {
-    if (!kv.second.ptr) continue;
+    if (!kv.second.ptr && !kv.second.ctrs) continue;
     cudaSetDevice(kv.first.first);
     cudaStreamSynchronize(kv.first.second);
-    cudaFree(kv.second.ptr);
+    if (kv.second.ptr) cudaFree(kv.second.ptr);
+    if (kv.second.ctrs) cudaFree(kv.second.ctrs);
   }
   g_ws.clear();
   for (auto& kv : g_stage) {

@@ -100,24 +100,87 @@ struct GemmMaps {
 };
 
 constexpr int kGemmBM = 128;
-constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;
 constexpr int kGemmStages = 4;
 
-size_t gemm_smem_bytes();
-cudaError_t launch_gemm(const GemmArgs& args, const GemmMaps& maps, int num_sms,
-                        cudaStream_t stream);
-// The same on CTA pairs (2-SM MMA, 256×256 tiles).  The A map's box must be
-// {64, 128} and the B map's {64, 64}, as for launch_gemm.
+// The same GEMM on CTA pairs (2-SM MMA, 256×256 tiles).  The A map's box
+// must be {64, 128} and the B map's {64, 64}.
 size_t gemm_pair_smem_bytes();
 cudaError_t launch_gemm_pair(const GemmArgs& args, const GemmMaps& maps, int num_sms,
                              cudaStream_t stream);
 
+// ------------------------------------------------------------------ chain
+// Several GEMMs C_p = Aop_p · Bop_p (+bias_p) in one persistent launch.  The
+// launch's tiles are the problems' tiles in order (within a problem, the
+// column tiles of one 128-row block are consecutive); CTA i takes tiles
+// i, i + grid, i + 2·grid, ...  A problem may signal a counter group: each
+// of its tiles, once stored, adds one arrival per epilogue warp to the
+// counter of its row block.  A later problem may wait on a group: before
+// loading operand a (the earlier problem's output) for a row block it waits
+// until that row block has `wait_count` arrivals.  Launches alternate
+// between two banks of counters; each launch zeroes the bank the next launch
+// will use (after the previous launch on the stream has finished), so the
+// counters need no reset from the host, even after an aborted launch.
+// Every dependency points to a lower tile index, which a running CTA owns,
+// so the waits always end (and are bounded regardless).
+constexpr int kChainMaxProbs = 12;
+constexpr int kChainMaxMaps = 32;
+
+struct ChainProblem {
+  int Mr, Nc, Kc;
+  int bn;            // tile columns: a multiple of 32 in [32, 256]
+  int tiles_m, tiles_n;
+  int tile_begin;    // index of the problem's first tile in the launch
+  int map_a, map_b;  // indices into ChainMaps
+  int map_c;         // store map of C (box 32 × 32, 64-byte swizzle), or -1:
+                     // C not TMA-able, stored by the epilogue threads
+  int a_col0;        // column of operand a where this problem's K range starts
+  __nv_bfloat16* c;
+  int64_t ldc;
+  const __nv_bfloat16* bias;
+  int wait_group;    // -1, or the counter group that gates operand a
+  int wait_count;    // arrivals that complete one row block of that group
+  int signal_group;  // -1, or the counter group this problem arrives on
+  int dep_a, dep_b;  // operand written by the previous launch on the stream
+};
+
+struct ChainArgs {
+  int n_prob;
+  int total_tiles;
+  ChainProblem p[kChainMaxProbs];
+  unsigned int* counters;       // this launch's bank: [group][ctr_stride], zero on entry
+  unsigned int* counters_next;  // the other bank, zeroed by this launch
+  int ctr_stride;
+  int n_counters;               // entries per bank
+  WaitCtl wait;
+  // The launch may start while the previous launch on the stream runs
+  // (programmatic dependent launch): operands flagged dep_a / dep_b are
+  // loaded only after griddepcontrol.wait, and every thread that writes
+  // global memory waits first too.
+  int pdl;
+  // Testing only: the producer withholds stage 0 of its first tile, so the
+  // MMA's bounded wait on it runs out (failure-detection test).
+  int withhold_first_stage;
+};
+
+struct ChainMaps {
+  // operand a: box {64, 128}; operand b: box {64, 64}; C: box {32, 32}
+  CUtensorMap m[kChainMaxMaps];
+};
+
+size_t chain_smem_bytes();
+cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& args, int grid,
+                         cudaStream_t stream);
+
 // Copy a [rows, cols] bf16 matrix with any 2-byte-aligned base and pitch lds
-// into dst (16-byte-aligned base, pitch ldd >= cols rounded up to 8).
+// into dst (16-byte-aligned base, pitch ldd >= cols rounded up to 8; the
+// columns from cols up to the next multiple of 8 are written as zero).
+// src_bytes is the byte extent of the source from its first element.  With
+// `dependent`, the launch may start while the previous launch on the stream
+// (which must not touch dst) still runs, and completes after it.
 cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_bytes,
                           __nv_bfloat16* dst, int64_t ldd, int64_t rows, int64_t cols,
-                          int num_sms, cudaStream_t stream);
+                          int num_sms, cudaStream_t stream, bool dependent = false);
 
 // Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0).
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,

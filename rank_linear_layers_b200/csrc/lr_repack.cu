@@ -6,86 +6,123 @@
 // TMA requires 16-byte-aligned row strides; a factor with r mod 8 != 0 has
 // none.  The GAC paper (§3.2, Table 3) shows what libraries do instead:
 // fall back to 2- or 1-element loads.  Here the misaligned matrix is read
-// once, at full width, with 16-byte loads (realigned in registers,
-// lr_load.cuh) and written once, aligned; the GEMM then runs its normal TMA
-// path.  Cost: one extra read and write of the matrix, bandwidth-bound.
+// once, at full width, with 16-byte loads and written once, aligned; the
+// GEMM then runs its normal TMA path.  Cost: one extra read of the matrix
+// from HBM and one write that stays in L2 until the GEMM has read it.
 #include <algorithm>
 
 #include "lr_internal.h"
-#include "lr_load.cuh"
 
 namespace lr {
 
 namespace {
 
-constexpr int kRepackWarps = 8;
-constexpr int kRepackU = 8;  // row segments in flight per warp
-constexpr int kRepackCtasPerSm = 2;
+constexpr int kRepackThreads = 256;
+constexpr int kRepackU = 4;  // destination chunks in flight per thread
 
-// The matrix is cut into 256-column segments of each row.  The grid's warps
-// are split into `segs` equal groups; the warps of group j copy segment j of
-// rows g, g + G, g + 2G, ... (G warps per group, g the warp's index in it),
-// through a rolling pipeline of kRepackU register slots: finishing row i
-// issues row i + kRepackU in its slot.  Only the start needs a division.
-__global__ void __launch_bounds__(kRepackWarps * 32) repack_rows_kernel(
-    const __nv_bfloat16* __restrict__ src, int64_t lds, uintptr_t lo, uintptr_t hi,
-    __nv_bfloat16* __restrict__ dst, int64_t ldd, int64_t rows, int64_t cols) {
+__device__ __forceinline__ uint4 ld_nc16(uintptr_t a) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(a));
+  return v;
+}
+
+// Bytes [sh, sh + 16) of the 32-byte window (lo, hi), sh even.
+__device__ __forceinline__ uint4 window16(const uint4& lo, const uint4& hi, uint32_t sh) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t o[5];
+  switch (sh >> 2) {
+    case 0: o[0] = w[0]; o[1] = w[1]; o[2] = w[2]; o[3] = w[3]; o[4] = w[4]; break;
+    case 1: o[0] = w[1]; o[1] = w[2]; o[2] = w[3]; o[3] = w[4]; o[4] = w[5]; break;
+    case 2: o[0] = w[2]; o[1] = w[3]; o[2] = w[4]; o[3] = w[5]; o[4] = w[6]; break;
+    default: o[0] = w[3]; o[1] = w[4]; o[2] = w[5]; o[3] = w[6]; o[4] = w[7]; break;
+  }
+  if (sh & 2u) {
+    return make_uint4(__byte_perm(o[0], o[1], 0x5432), __byte_perm(o[1], o[2], 0x5432),
+                      __byte_perm(o[2], o[3], 0x5432), __byte_perm(o[3], o[4], 0x5432));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One thread per 16-byte destination chunk (row k, elements 8j .. 8j+7):
+// the chunk's source bytes span at most two aligned 16-byte granules of the
+// source, both of which hold an element of the matrix (the first holds the
+// chunk's first element; the second is read only if it starts before the end
+// of the source buffer), so no load leaves the buffer's pages.  Elements
+// past the row's end are written as zero.
+__global__ void __launch_bounds__(kRepackThreads) repack_chunks_kernel(
+    const __nv_bfloat16* __restrict__ src, int64_t lds, uintptr_t hi,
+    __nv_bfloat16* __restrict__ dst, int64_t ldd, uint32_t cols, uint32_t cpr, uint32_t total) {
   griddep_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int segs = static_cast<int>((cols + 255) / 256);
-  const int w = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  const int W = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
-  const int G = W / segs;  // warps per segment (the launch makes it >= 1)
-  if (w >= G * segs) return;
-  const int seg = w % segs, g = w / segs;
-  const int64_t c0 = static_cast<int64_t>(seg) * 256;
-  const int nv = static_cast<int>(std::min<int64_t>(256, cols - c0));
-  const int64_t mine = (rows > g) ? (rows - g + G - 1) / G : 0;  // rows of this warp
-  const __nv_bfloat16* s0 = src + static_cast<int64_t>(g) * lds + c0;
-  const int64_t sstep = static_cast<int64_t>(G) * lds;
-  __nv_bfloat16* d0 = dst + static_cast<int64_t>(g) * ldd + c0;
-  const int64_t dstep = static_cast<int64_t>(G) * ldd;
-
-  uint4 cur[kRepackU], ext[kRepackU];
-#pragma unroll
-  for (int u = 0; u < kRepackU; ++u)
-    seg16_issue(s0 + u * sstep, lane, 32, u < mine ? nv : 0, lo, hi, cur[u], ext[u]);
-  for (int64_t i0 = 0; i0 < mine; i0 += kRepackU) {
+  const uint32_t stride = gridDim.x * kRepackThreads;
+  for (uint32_t q0 = blockIdx.x * kRepackThreads + threadIdx.x; q0 < total;
+       q0 += kRepackU * stride) {
+    uint4 lo[kRepackU], hi2[kRepackU];
+    uint32_t shift[kRepackU];
 #pragma unroll
     for (int u = 0; u < kRepackU; ++u) {
-      const int64_t i = i0 + u;
-      if (i >= mine) break;
-      const __nv_bfloat16* sp = s0 + i * sstep;
-      const uint4 v = seg16_finish(cur[u], ext[u], seg_shift(sp), lane, 32, nv);
-      // Refill the slot with row i + U before storing this one.
-      seg16_issue(sp + kRepackU * sstep, lane, 32, i + kRepackU < mine ? nv : 0, lo, hi, cur[u],
-                  ext[u]);
-      const int c = 8 * lane;
-      if (c < nv) {
-        // dst rows are 16-byte aligned and c0 + c is a multiple of 8: the
-        // chunk is aligned; elements past nv are zero, and the pitch covers
-        // them (ldd >= cols rounded up to 8).
-        *reinterpret_cast<uint4*>(d0 + i * dstep + c) = v;
+      const uint32_t q = q0 + u * stride;
+      if (q < total) {
+        const uint32_t k = q / cpr, j = q - k * cpr;
+        const uintptr_t p = reinterpret_cast<uintptr_t>(src + static_cast<int64_t>(k) * lds + 8 * j);
+        const uintptr_t a = p & ~static_cast<uintptr_t>(15);
+        shift[u] = static_cast<uint32_t>(p & 15u);
+        lo[u] = ld_nc16(a);
+        hi2[u] = (shift[u] != 0u && a + 16 < hi) ? ld_nc16(a + 16) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRepackU; ++u) {
+      const uint32_t q = q0 + u * stride;
+      if (q < total) {
+        const uint32_t k = q / cpr, j = q - k * cpr;
+        uint4 v = window16(lo[u], hi2[u], shift[u]);
+        const int valid = static_cast<int>(cols) - static_cast<int>(8 * j);
+        if (valid < 8) {
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (e >= valid) w[e >> 1] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+          v = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(k) * ldd + 8 * j) = v;
       }
     }
   }
+  // A later repack of the same call may start early (programmatic dependent
+  // launch); finishing only after this one's predecessor keeps completion in
+  // stream order.
+  griddep_wait();
 }
 
 }  // namespace
 
 cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_bytes,
                           __nv_bfloat16* dst, int64_t ldd, int64_t rows, int64_t cols,
-                          int num_sms, cudaStream_t stream) {
+                          int num_sms, cudaStream_t stream, bool dependent) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
-  const uintptr_t lo = reinterpret_cast<uintptr_t>(src);
-  // Enough warps that every segment gets at least one and the SMs fill.
-  const int64_t segs = (cols + 255) / 256;
-  const int64_t warps_wanted = std::max<int64_t>(segs, std::min<int64_t>(
-      segs * rows, static_cast<int64_t>(num_sms) * kRepackCtasPerSm * kRepackWarps));
-  const int blocks = static_cast<int>(std::max<int64_t>(1, (warps_wanted + kRepackWarps - 1) / kRepackWarps));
-  repack_rows_kernel<<<blocks, kRepackWarps * 32, 0, stream>>>(src, lds, lo, lo + src_bytes, dst,
-                                                               ldd, rows, cols);
-  return cudaGetLastError();
+  const int64_t cpr = (cols + 7) / 8;
+  const int64_t total = rows * cpr;
+  if (total > 0xFFFFFFFFll - static_cast<int64_t>(num_sms) * 8 * kRepackThreads * kRepackU)
+    return cudaErrorInvalidValue;
+  const uintptr_t hi = reinterpret_cast<uintptr_t>(src) + src_bytes;
+  const int64_t per_cta = static_cast<int64_t>(kRepackThreads) * kRepackU;
+  const int blocks = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>((total + per_cta - 1) / per_cta,
+                                             static_cast<int64_t>(num_sms) * 8)));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(kRepackThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, repack_chunks_kernel, src, lds, hi, dst, ldd,
+                            static_cast<uint32_t>(cols), static_cast<uint32_t>(cpr),
+                            static_cast<uint32_t>(total));
 }
 
 }  // namespace lr

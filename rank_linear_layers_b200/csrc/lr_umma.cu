@@ -1,4 +1,4 @@
-// lr_umma.cu — tcgen05 (5th-generation tensor core) GEMM tile engine for the
+// lr_umma.cu — tcgen05 (5th-generation tensor core) GEMM engine for the
 // prefill path of Y = (X·A)·B (+bias).
 //
 //   GEMM1:  T [M, r] = X [M, K] · A [K, r]        (T written once, bf16)
@@ -8,15 +8,20 @@
 // Bop row-major (N contiguous: "MN-major"); the tensor core reads both
 // layouts from shared memory directly, so no operand is transposed.
 //
-// Structure (one persistent CTA per SM, warp-specialised, 192 threads):
+// umma_chain_kernel runs a list of such GEMMs in one persistent launch (one
+// CTA per SM, warp-specialised, 192 threads):
 //   warps 0-3  epilogue: TMEM -> registers -> +bias -> bf16 -> global
-//   warp 4     one elected thread issues tcgen05.mma (128×256×16 per issue)
+//   warp 4     one elected thread issues tcgen05.mma (128 × bn × 16 per issue)
 //   warp 5     one thread issues the TMA tile loads (128-byte swizzle)
 // A 4-stage shared-memory ring (mbarrier full/empty pairs) feeds the MMA;
 // two TMEM accumulators (2 × 256 fp32 columns) let the epilogue of one tile
-// overlap the main loop of the next.  Operands must have 16-byte-aligned
-// bases and row pitches (TMA's rule); the host realigns any that do not
-// (lr_repack.cu) before launching.
+// overlap the main loop of the next.  Each problem has its own tile width
+// bn (a multiple of 16 up to 256), chosen on the host so that the launch's
+// tiles spread evenly over the SMs.  GEMM2's tiles of a 128-row block wait
+// (bounded) for GEMM1's tiles of that block, so the two contractions share
+// one launch and GEMM2 starts row block by row block.  Operands must have
+// 16-byte-aligned bases and row pitches (TMA's rule); the host realigns any
+// that do not (lr_repack.cu) before launching.
 //
 // Ragged edges cost no padding on the host: TMA zero-fills out-of-bounds
 // rows and columns, the last K block issues only the 16-deep MMA steps it
@@ -33,19 +38,25 @@ namespace lr {
 namespace {
 
 constexpr int BM = kGemmBM;
-constexpr int BN = kGemmBN;
 constexpr int BK = kGemmBK;
 constexpr int STAGES = kGemmStages;
-constexpr int A_STAGE = BM * BK * 2;  // 16 KB
-constexpr int B_STAGE = BK * BN * 2;  // 32 KB
+constexpr int MAX_BN = 256;
+constexpr int A_STAGE = BM * BK * 2;      // 16 KB
+constexpr int B_STAGE = BK * MAX_BN * 2;  // 32 KB
 constexpr int STAGE = A_STAGE + B_STAGE;
-constexpr int B_ATOM = BK * 128;      // one 64-column MN-major atom column: 8 KB
+constexpr int B_ATOM = BK * 128;          // one 64-column MN-major atom column: 8 KB
 constexpr int EPI_WARPS = 4;
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
-constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t TMEM_COLS = 2 * MAX_BN;
+// Epilogue staging for TMA stores: per epilogue warp four 32-row × 32-column
+// bf16 boxes (64-byte rows, 64-byte swizzle), used in rotation.
+constexpr int EPI_BOX = 32 * 64;
+constexpr int EPI_BOXES = 4;
+constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BOXES * EPI_BOX;  // 32 KB
 
-constexpr unsigned kWhereProducer = 1, kWhereMma = 3, kWhereMmaAcc = 4, kWhereEpilogue = 5;
+constexpr unsigned kWhereProducer = 1, kWhereMma = 3, kWhereMmaAcc = 4, kWhereEpilogue = 5,
+                   kWhereDependency = 6;
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
                                                 unsigned long long limit_ns) {
@@ -56,27 +67,23 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
   return true;
 }
 
-struct Smem {
-  uint8_t* base;  // 1024-aligned
-  __device__ uint8_t* a(int s) const { return base + s * STAGE; }
-  __device__ uint8_t* b(int s) const { return base + s * STAGE + A_STAGE; }
-};
-
-__device__ __forceinline__ void store_chunk(const GemmArgs& g, int row, int col0,
+// Store 32 accumulator columns [col0, col0 + 32) of one output row, columns
+// at or past `cend` skipped.
+__device__ __forceinline__ void store_chunk(__nv_bfloat16* c, int64_t ldc,
+                                            const __nv_bfloat16* bias, int row, int col0, int cend,
                                             const uint32_t (&v)[32], bool vec_ok) {
-  if (row >= g.Mr) return;
   float f[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-  if (g.bias) {
+  if (bias) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const int c = col0 + i;
-      if (c < g.Nc) f[i] += __bfloat162float(g.bias[c]);
+      const int col = col0 + i;
+      if (col < cend) f[i] += __bfloat162float(bias[col]);
     }
   }
-  __nv_bfloat16* dst = g.c + static_cast<int64_t>(row) * g.ldc + col0;
-  if (vec_ok && col0 + 32 <= g.Nc) {
+  __nv_bfloat16* dst = c + static_cast<int64_t>(row) * ldc + col0;
+  if (vec_ok && col0 + 32 <= cend) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 w;
@@ -89,24 +96,54 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int row, int col0
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-      if (col0 + i < g.Nc) dst[i] = __float2bfloat16_rn(f[i]);
+      if (col0 + i < cend) dst[i] = __float2bfloat16_rn(f[i]);
   }
 }
 
 constexpr int kGemmThreads = 6 * 32;
 
+__device__ __forceinline__ int find_problem(const ChainArgs& g, int tile) {
+  int i = 0;
+  while (i + 1 < g.n_prob && tile >= g.p[i + 1].tile_begin) ++i;
+  return i;
+}
+
+// Wait until row block m_blk of counter group `grp` has `count` arrivals.
+// Bounded; on a timeout it records the error.
+__device__ bool wait_rows_ready(const ChainArgs& g, int grp, int m_blk, int count) {
+  const unsigned int* ctr = g.counters + static_cast<int64_t>(grp) * g.ctr_stride + m_blk;
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_u32(ctr) >= static_cast<unsigned int>(count)) break;
+    if (it == 0) t0 = global_ns();
+    __nanosleep(64);
+    if ((it & 15u) == 15u) {
+      if (aborted(g.wait)) return false;
+      if (global_ns() - t0 > g.wait.timeout_ns) {
+        record_timeout(g.wait, kWhereDependency);
+        return false;
+      }
+    }
+  }
+  // Order the acquire before this thread's TMA (async-proxy) reads.
+  fence_proxy_async_global();
+  return true;
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    umma_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
-                     const __grid_constant__ CUtensorMap map_b, const GemmArgs g) {
+    umma_chain_kernel(const __grid_constant__ ChainMaps maps, const __grid_constant__ ChainArgs g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  Smem sm{smem_raw + (((raw + 1023u) & ~1023u) - raw)};
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm.base + STAGES * STAGE);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* epi_stage = base + STAGES * STAGE;  // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_stage + EPI_STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* fin = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
+  auto stage_a = [&](int s) { return base + s * STAGE; };
+  auto stage_b = [&](int s) { return base + s * STAGE + A_STAGE; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -128,17 +165,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == TMA_WARP && lane == 0) {
-    tma_prefetch_desc(&map_a);
-    tma_prefetch_desc(&map_b);
+  if (warp == TMA_WARP && lane == 0 && blockIdx.x < g.total_tiles) {
+    const ChainProblem& P = g.p[find_problem(g, blockIdx.x)];
+    tma_prefetch_desc(&maps.m[P.map_a]);
+    tma_prefetch_desc(&maps.m[P.map_b]);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int num_tiles = g.tiles_m * g.tiles_n;
-  const int num_kb = (g.Kc + BK - 1) / BK;
   // Producer bookkeeping for a clean exit after a timeout.
   int issued_phase[STAGES];
 #pragma unroll
@@ -147,52 +183,89 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == TMA_WARP) {
     if (lane == 0) {
-      auto load_a = [&](int s, int kb, int m_blk) {
-        tma_load_2d(sm.a(s), &map_a, &full[s], kb * BK, m_blk * BM);
-      };
-      auto load_b = [&](int s, int kb, int n_blk) {
-#pragma unroll
-        for (int c = 0; c < BN / 64; ++c)
-          tma_load_2d(sm.b(s) + c * B_ATOM, &map_b, &full[s], n_blk * BN + c * 64, kb * BK);
-      };
-      // Under programmatic dependent launch, fill the first stages with the
-      // operands the previous launch does not write, wait for it, then add
-      // the rest.  The first STAGES stages are free on entry.
-      int pre = 0;
-      if (g.pdl) {
-        const int tile = blockIdx.x;
-        if (tile < num_tiles) {
-          const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
-          pre = num_kb < STAGES ? num_kb : STAGES;
-          const int first = g.withhold_first_stage ? 1 : 0;
-          for (int kb = first; kb < pre; ++kb) {
-            mbar_arrive_expect_tx(&full[kb], A_STAGE + B_STAGE);
-            if (!g.dep_a) load_a(kb, kb, m_blk);
-            if (!g.dep_b) load_b(kb, kb, n_blk);
+      int s = 0;
+      uint32_t ph = 0;
+      bool first = true;
+      for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x) {
+        const ChainProblem& P = g.p[find_problem(g, tile)];
+        const int local = tile - P.tile_begin;
+        const int m_blk = local / P.tiles_n, n_blk = local - m_blk * P.tiles_n;
+        const int num_kb = (P.Kc + BK - 1) / BK;
+        const int nbox = (P.bn + 63) / 64;
+        const uint32_t bytes = A_STAGE + nbox * B_ATOM;
+        const CUtensorMap* ma = &maps.m[P.map_a];
+        const CUtensorMap* mb = &maps.m[P.map_b];
+        auto load_a = [&](int st, int kb) {
+          tma_load_2d(stage_a(st), ma, &full[st], P.a_col0 + kb * BK, m_blk * BM);
+        };
+        auto load_b = [&](int st, int kb) {
+          for (int c = 0; c < nbox; ++c)
+            tma_load_2d(stage_b(st) + c * B_ATOM, mb, &full[st], n_blk * P.bn + c * 64, kb * BK);
+        };
+        const bool gated_a = P.dep_a || P.wait_group >= 0;
+        const bool gated_b = P.dep_b;
+        int kb0 = 0;
+        if (first) {
+          first = false;
+          if (g.pdl) {
+            // Fill the first (free) stages with operands nothing earlier
+            // writes, wait for the previous launch, then add the rest.
+            const int pre = num_kb < STAGES ? num_kb : STAGES;
+            const int skip = g.withhold_first_stage ? 1 : 0;
+            for (int kb = skip; kb < pre; ++kb) {
+              mbar_arrive_expect_tx(&full[kb], bytes);
+              if (!gated_a) load_a(kb, kb);
+              if (!gated_b) load_b(kb, kb);
+              issued_phase[kb] = 0;
+            }
+            griddep_wait();
+            if (P.wait_group >= 0 && !wait_rows_ready(g, P.wait_group, m_blk, P.wait_count)) {
+              ok = false;
+              break;
+            }
+            for (int kb = skip; kb < pre; ++kb) {
+              if (gated_a) load_a(kb, kb);
+              if (gated_b) load_b(kb, kb);
+            }
+            kb0 = pre;
+            s = pre % STAGES;
+            ph = (pre == STAGES) ? 1u : 0u;
           }
-          griddep_wait();
-          for (int kb = first; kb < pre; ++kb) {
-            if (g.dep_a) load_a(kb, kb, m_blk);
-            if (g.dep_b) load_b(kb, kb, n_blk);
-            issued_phase[kb] = 0;
-          }
-        } else {
-          griddep_wait();
         }
-      }
-      int s = pre % STAGES;
-      uint32_t ph = (pre == STAGES) ? 1u : 0u;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
-        for (int kb = (tile == static_cast<int>(blockIdx.x)) ? pre : 0; kb < num_kb; ++kb) {
+        if (kb0 == 0 && P.wait_group >= 0) {
+          // Operand b does not depend on the rows being waited for: put it
+          // into the first stages, then wait, then add operand a.
+          const int pre = num_kb < STAGES ? num_kb : STAGES;
+          const int s0 = s;
+          for (int kb = 0; kb < pre && ok; ++kb) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereProducer)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], bytes);
+            load_b(s, kb);
+            issued_phase[s] = static_cast<int>(ph);
+            if (++s == STAGES) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+          if (!ok || !wait_rows_ready(g, P.wait_group, m_blk, P.wait_count)) {
+            ok = false;
+            break;
+          }
+          for (int kb = 0; kb < pre; ++kb) load_a((s0 + kb) % STAGES, kb);
+          kb0 = pre;
+        }
+        for (int kb = kb0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, g.wait, kWhereProducer)) {
             ok = false;
             break;
           }
           if (!(g.withhold_first_stage && kb == 0 && tile == static_cast<int>(blockIdx.x))) {
-            mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
-            load_a(s, kb, m_blk);
-            load_b(s, kb, n_blk);
+            mbar_arrive_expect_tx(&full[s], bytes);
+            load_a(s, kb);
+            load_b(s, kb);
             issued_phase[s] = static_cast<int>(ph);
           }
           if (++s == STAGES) {
@@ -203,11 +276,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == MMA_WARP) {
-    const uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
     int s = 0;
     uint32_t ph = 0;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+    for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x, ++it) {
+      const ChainProblem& P = g.p[find_problem(g, tile)];
+      const int num_kb = (P.Kc + BK - 1) / BK;
+      const uint32_t idesc = idesc_bf16_f32(BM, P.bn, false, true);
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
       if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait, kWhereMmaAcc)) {
@@ -215,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MAX_BN);
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&full[s], ph, g.wait, kWhereMma)) {
           ok = false;
@@ -223,10 +298,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         if (lane == 0) {
-          const int krem = g.Kc - kb * BK;
+          const int krem = P.Kc - kb * BK;
           const int nk = krem >= BK ? BK / 16 : (krem + 15) / 16;
-          const uint32_t a0 = smem_u32(sm.a(s));
-          const uint32_t b0 = smem_u32(sm.b(s));
+          const uint32_t a0 = smem_u32(stage_a(s));
+          const uint32_t b0 = smem_u32(stage_b(s));
           for (int kk = 0; kk < nk; ++kk) {
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b0 + kk * 2048, B_ATOM, 1024);
@@ -245,10 +320,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
     }
   } else if (warp < EPI_WARPS) {
-    const bool vec_ok = ((reinterpret_cast<uintptr_t>(g.c) & 15u) == 0) && ((g.ldc & 7) == 0);
+    // Under programmatic dependent launch, write nothing before the previous
+    // launch on the stream has finished (it may still read these buffers).
+    griddep_wait();
+    if (blockIdx.x == 0)  // the next launch's counter bank (the previous launch used it)
+      for (int i = threadIdx.x; i < g.n_counters; i += EPI_WARPS * 32) g.counters_next[i] = 0u;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-      const int m_blk = tile % g.tiles_m, n_blk = tile / g.tiles_m;
+    int epi_box = 0;  // boxes this warp has staged (rotating buffers)
+    for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x, ++it) {
+      const ChainProblem& P = g.p[find_problem(g, tile)];
+      const int local = tile - P.tile_begin;
+      const int m_blk = local / P.tiles_n, n_blk = local - m_blk * P.tiles_n;
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
       if (!mbar_wait(&tfull[acc], aph, g.wait, kWhereEpilogue)) {
@@ -256,22 +338,94 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = m_blk * BM + warp * 32 + lane;
+      const bool vec_ok =
+          ((reinterpret_cast<uintptr_t>(P.c) & 15u) == 0) && ((P.ldc & 7) == 0);
+      const int row0 = m_blk * BM + warp * 32;
+      const int row = row0 + lane;
+      const int n0 = n_blk * P.bn;
+      const int cend = min(P.Nc, n0 + P.bn);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+                             static_cast<uint32_t>(acc * MAX_BN);
+      const CUtensorMap* mc = P.map_c >= 0 ? &maps.m[P.map_c] : nullptr;
+      // One 32-column chunk: bf16 rounding (+bias) and the store.
+      auto emit = [&](const uint32_t (&v)[32], int c) {
+        const int col0 = n0 + c * 32;
+        if (mc) {
+          // Stage the warp's 32 × 32 box in shared memory (row = lane,
+          // 16-byte chunks swizzled so that the warp's writes hit every bank
+          // once per 128 bytes) and let TMA write it out with full-line
+          // stores; the map clips rows >= Mr and columns >= Nc.
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float lo = __uint_as_float(v[2 * i]), hi = __uint_as_float(v[2 * i + 1]);
+            if (P.bias) {
+              const int cl = col0 + 2 * i;
+              if (cl < cend) lo += __bfloat162float(P.bias[cl]);
+              if (cl + 1 < cend) hi += __bfloat162float(P.bias[cl + 1]);
+            }
+            w[i] = pack_bf16x2(lo, hi);
+          }
+          uint8_t* box = epi_stage + (warp * EPI_BOXES + (epi_box % EPI_BOXES)) * EPI_BOX;
+          if (epi_box >= EPI_BOXES) {
+            // The store that used this box last has read it.
+            if (lane == 0) bulk_wait_group_read<EPI_BOXES - 1>();
+            __syncwarp();
+          }
+          const int sw = (lane >> 1) & 3;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ sw) << 4)) =
+                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(mc, box, col0, row0);
+            bulk_commit_group();
+          }
+          ++epi_box;
+        } else if (row < P.Mr) {
+          store_chunk(P.c, P.ldc, P.bias, row, col0, cend, v, vec_ok);
+        }
+      };
+      // Chunks alternate between two register sets: the TMEM load of chunk
+      // c + 1 is in flight while chunk c is rounded and stored.
+      const int nch = (min(P.bn, cend - n0) + 31) / 32;
+      uint32_t va[32], vb[32];
+      tmem_ld_32x32b_x32(t_row, va);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = n_blk * BN + c * 32;
-        if (col0 >= g.Nc) break;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
-        tmem_ld_wait();
-        store_chunk(g, row, col0, v, vec_ok);
+      for (int c = 0; c < nch; c += 2) {
+        tmem_ld_wait(va);
+        if (c + 1 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * 32), vb);
+        emit(va, c);
+        if (c + 1 < nch) {
+          tmem_ld_wait(vb);
+          if (c + 2 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * 32), va);
+          emit(vb, c + 1);
+        }
       }
       tc_fence_before();
+      if (P.signal_group >= 0) {
+        // This warp's rows of the tile are written: make them visible to the
+        // TMA loads of other CTAs, then count the arrival.
+        if (mc) {
+          if (lane == 0) bulk_wait_group<0>();
+        } else {
+          fence_proxy_async_global();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          fence_proxy_async_global();
+          __threadfence();
+          atomicAdd(g.counters + static_cast<int64_t>(P.signal_group) * g.ctr_stride + m_blk, 1u);
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    // The staged boxes must stay in place until TMA has read them.
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   // Teardown.  Every wait above is bounded, so every thread gets here.
@@ -283,7 +437,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == TMA_WARP && lane == 0 && !ok) {
     // After a timeout: let any TMA load still in flight land before exit.
     for (int s = 0; s < STAGES; ++s)
-      if (issued_phase[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_phase[s]), 1000000ull);
+      if (issued_phase[s] >= 0)
+        mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_phase[s]), 1000000ull);
   }
   tc_fence_before();
   __syncthreads();
@@ -406,7 +561,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * P_BN);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[s], ph, g.wait, kWhereMma)) {
             ok = false;
@@ -451,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int row = m_blk * P_BM + static_cast<int>(rank) * 128 + warp * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+                             static_cast<uint32_t>(acc * P_BN);
 #pragma unroll 1
       for (int c = 0; c < P_BN / 32; ++c) {
         const int col0 = n_blk * P_BN + c * 32;
@@ -459,7 +614,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
-        store_chunk(g, row, col0, v, vec_ok);
+        if (row < g.Mr) store_chunk(g.c, g.ldc, g.bias, row, col0, g.Nc, v, vec_ok);
       }
       tc_fence_before();
       __syncwarp();
@@ -498,8 +653,9 @@ __global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64
 
 }  // namespace
 
-size_t gemm_smem_bytes() {
-  return 1024 + static_cast<size_t>(STAGES) * STAGE + (2 * STAGES + 5) * sizeof(uint64_t) + 16;
+size_t chain_smem_bytes() {
+  return 1024 + static_cast<size_t>(STAGES) * STAGE + EPI_STAGE_BYTES +
+         (2 * STAGES + 5) * sizeof(uint64_t) + 16;
 }
 
 size_t gemm_pair_smem_bytes() {
@@ -519,15 +675,14 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, const GemmMaps& maps, int num_sm
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,
-                        cudaStream_t stream) {
-  const size_t smem = gemm_smem_bytes();
+cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid,
+                         cudaStream_t stream) {
+  const size_t smem = chain_smem_bytes();
   cudaError_t e =
-      ensure_max_smem(reinterpret_cast<const void*>(umma_gemm_kernel), static_cast<int>(smem));
+      ensure_max_smem(reinterpret_cast<const void*>(umma_chain_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int tiles = g.tiles_m * g.tiles_n;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(std::max(1, std::min(tiles, num_sms)));
+  cfg.gridDim = dim3(std::max(1, grid));
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -536,7 +691,7 @@ cudaError_t launch_gemm(const GemmArgs& g, const GemmMaps& maps, int num_sms,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = g.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel, maps.a, maps.b, g);
+  return cudaLaunchKernelEx(&cfg, umma_chain_kernel, maps, g);
 }
 
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,

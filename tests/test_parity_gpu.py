@@ -102,6 +102,30 @@ def test_pair_and_single_sm_kernels_agree(lr, M, K, r, N):
     compare(Y1[rows], Yr, "single-SM kernel")
 
 
+@pytest.mark.parametrize("bn", [32, 64, 96, 128, 160, 192, 224, 256])
+def test_prefill_forced_tile_width(lr, bn):
+    """Every tile width the planner may pick, on a ragged shape (odd K, r, N;
+    partial 64-column atoms when bn is not a multiple of 64; Y rows not
+    16-byte aligned, so Y takes the per-thread stores and T the TMA stores)."""
+    p = lrgen.lowrank_problem(300, 333, 257, 517, seed=bn, bias=True)
+    lr.set_tile_n(bn)
+    try:
+        Y = run_gpu(lr, p, lr.PATH_PREFILL)
+    finally:
+        lr.set_tile_n(0)
+    compare(Y, ref(p), f"prefill bn={bn}")
+
+
+@pytest.mark.parametrize("r", [1024, 1025, 1032])
+def test_prefill_tile_plan_around_1024(lr, r):
+    """M = K = N = 4096 around r = 1024, where the chosen tile widths change
+    (sampled rows, computed one by one by the oracle)."""
+    p = lrgen.lowrank_problem(4096, 4096, r, 4096, seed=r)
+    Y = run_gpu(lr, p)
+    rows = np.concatenate([np.random.default_rng(r).choice(4096, 40, replace=False), [0, 4095]])
+    compare(Y[rows], ref(p, rows=rows), f"r={r} sampled rows")
+
+
 def test_decode_and_prefill_agree_at_m16(lr):
     p = lrgen.lowrank_problem(16, 512, 300, 640, seed=3, bias=True)
     Yd = run_gpu(lr, p, lr.PATH_DECODE)
