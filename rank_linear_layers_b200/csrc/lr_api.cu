@@ -60,10 +60,9 @@ struct MapKey {
   const void* ptr;
   uint64_t inner, outer, stride;
   uint32_t box_inner, box_outer;
-  int swizzle;
   bool operator<(const MapKey& o) const {
-    return std::tie(ptr, inner, outer, stride, box_inner, box_outer, swizzle) <
-           std::tie(o.ptr, o.inner, o.outer, o.stride, o.box_inner, o.box_outer, o.swizzle);
+    return std::tie(ptr, inner, outer, stride, box_inner, box_outer) <
+           std::tie(o.ptr, o.inner, o.outer, o.stride, o.box_inner, o.box_outer);
   }
 };
 std::map<MapKey, CUtensorMap> g_maps;
@@ -110,14 +109,12 @@ lr_status get_encoder() {
   return LR_OK;
 }
 
-// 2-D bf16 tensor map (128-byte swizzle unless `swizzle64`), out-of-bounds
-// elements read as zero (loads) or are not written (stores).
+// 2-D bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
 lr_status tensor_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t outer,
-                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer,
-                     bool swizzle64 = false) {
+                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer) {
   lr_status st = get_encoder();
   if (st != LR_OK) return st;
-  MapKey key{ptr, inner, outer, row_stride_elems, box_inner, box_outer, swizzle64 ? 64 : 128};
+  MapKey key{ptr, inner, outer, row_stride_elems, box_inner, box_outer};
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_maps.find(key);
@@ -132,8 +129,7 @@ lr_status tensor_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_last_cuda_error = static_cast<int>(r);
@@ -337,17 +333,8 @@ lr_status chain_problem(ChainBuild& cb, int map_a, int a_col0, int map_b, int64_
                         int64_t Kc, void* c, int64_t ldc, const void* bias, int wait_group,
                         int signal_group, bool dep_a, bool dep_b) {
   if (cb.args.n_prob >= kChainMaxProbs) return LR_ERR_UNSUPPORTED;
-  // C through TMA stores when its base and pitch allow, else plain stores.
-  int map_c = -1;
-  if (tma_ok(c, ldc) && cb.n_maps < kChainMaxMaps) {
-    lr_status st = tensor_map(&cb.maps.m[cb.n_maps], c, static_cast<uint64_t>(Nc),
-                              static_cast<uint64_t>(Mr), static_cast<uint64_t>(ldc), 32, 32, true);
-    if (st != LR_OK) return st;
-    map_c = cb.n_maps++;
-  }
   ChainProblem& P = cb.args.p[cb.args.n_prob++];
   P = ChainProblem{};
-  P.map_c = map_c;
   P.Mr = static_cast<int>(Mr);
   P.Nc = static_cast<int>(Nc);
   P.Kc = static_cast<int>(Kc);
@@ -497,7 +484,7 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
     if (P.wait_group < 0) continue;
     P.wait_count = 0;
     for (int j = 0; j < i; ++j)
-      if (a.p[j].signal_group == P.wait_group) P.wait_count += 4 * a.p[j].tiles_n;
+      if (a.p[j].signal_group == P.wait_group) P.wait_count += kChainEpiWarps * a.p[j].tiles_n;
   }
   a.total_tiles = static_cast<int>(total);
   if (total == 0) return LR_OK;

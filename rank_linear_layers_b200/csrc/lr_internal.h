@@ -114,8 +114,8 @@ cudaError_t launch_gemm_pair(const GemmArgs& args, const GemmMaps& maps, int num
 // launch's tiles are the problems' tiles in order (within a problem, the
 // column tiles of one 128-row block are consecutive); CTA i takes tiles
 // i, i + grid, i + 2·grid, ...  A problem may signal a counter group: each
-// of its tiles, once stored, adds one arrival per epilogue warp to the
-// counter of its row block.  A later problem may wait on a group: before
+// of its tiles, once stored, adds one arrival per epilogue warp
+// (kChainEpiWarps) to the counter of its row block.  A later problem may wait on a group: before
 // loading operand a (the earlier problem's output) for a row block it waits
 // until that row block has `wait_count` arrivals.  Launches alternate
 // between two banks of counters; each launch zeroes the bank the next launch
@@ -124,7 +124,8 @@ cudaError_t launch_gemm_pair(const GemmArgs& args, const GemmMaps& maps, int num
 // Every dependency points to a lower tile index, which a running CTA owns,
 // so the waits always end (and are bounded regardless).
 constexpr int kChainMaxProbs = 12;
-constexpr int kChainMaxMaps = 32;
+constexpr int kChainEpiWarps = 8;  // arrivals per finished tile
+constexpr int kChainMaxMaps = 24;
 
 struct ChainProblem {
   int Mr, Nc, Kc;
@@ -132,8 +133,6 @@ struct ChainProblem {
   int tiles_m, tiles_n;
   int tile_begin;    // index of the problem's first tile in the launch
   int map_a, map_b;  // indices into ChainMaps
-  int map_c;         // store map of C (box 32 × 32, 64-byte swizzle), or -1:
-                     // C not TMA-able, stored by the epilogue threads
   int a_col0;        // column of operand a where this problem's K range starts
   __nv_bfloat16* c;
   int64_t ldc;
@@ -164,8 +163,7 @@ struct ChainArgs {
 };
 
 struct ChainMaps {
-  // operand a: box {64, 128}; operand b: box {64, 64}; C: box {32, 32}
-  CUtensorMap m[kChainMaxMaps];
+  CUtensorMap m[kChainMaxMaps];  // operand a: box {64, 128}; operand b: box {64, 64}
 };
 
 size_t chain_smem_bytes();

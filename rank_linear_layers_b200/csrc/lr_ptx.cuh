@@ -124,35 +124,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, uintptr_t gsrc, uint32
       : "memory");
 }
 
-// TMA tile store shared -> global (bulk-group completion); the tensor map's
-// bounds clip rows and columns outside the tensor.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src,
-                                             int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(smem_src)), "r"(x), "r"(y)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N of this thread's committed bulk groups still read
-// their shared-memory source.
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until at most N of this thread's committed bulk groups are pending
-// (their writes performed).
-template <int N>
-__device__ __forceinline__ void bulk_wait_group() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -45,15 +45,22 @@ constexpr int A_STAGE = BM * BK * 2;      // 16 KB
 constexpr int B_STAGE = BK * MAX_BN * 2;  // 32 KB
 constexpr int STAGE = A_STAGE + B_STAGE;
 constexpr int B_ATOM = BK * 128;          // one 64-column MN-major atom column: 8 KB
+// CTA-pair kernel roles.
 constexpr int EPI_WARPS = 4;
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
+// Chain kernel roles: two epilogue warps per 32-lane quarter of TMEM (warp w
+// reads lanes 32·(w mod 4) and takes every other 32-column chunk), then the
+// MMA warp and the TMA warp.
+constexpr int C_EPI_WARPS = kChainEpiWarps;
+constexpr int C_MMA_WARP = C_EPI_WARPS;
+constexpr int C_TMA_WARP = C_EPI_WARPS + 1;
+constexpr int kChainThreads = (C_EPI_WARPS + 2) * 32;
 constexpr uint32_t TMEM_COLS = 2 * MAX_BN;
-// Epilogue staging for TMA stores: per epilogue warp four 32-row × 32-column
-// bf16 boxes (64-byte rows, 64-byte swizzle), used in rotation.
+// Epilogue transpose buffers: per epilogue warp two 32-row × 32-column bf16
+// boxes (64-byte rows), used alternately.
 constexpr int EPI_BOX = 32 * 64;
-constexpr int EPI_BOXES = 4;
-constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BOXES * EPI_BOX;  // 32 KB
+constexpr int EPI_STAGE_BYTES = kChainEpiWarps * 2 * EPI_BOX;  // 32 KB
 
 constexpr unsigned kWhereProducer = 1, kWhereMma = 3, kWhereMmaAcc = 4, kWhereEpilogue = 5,
                    kWhereDependency = 6;
@@ -68,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
 }
 
 // Store 32 accumulator columns [col0, col0 + 32) of one output row, columns
-// at or past `cend` skipped.
+// at or past `cend` skipped (the CTA-pair kernel's epilogue).
 __device__ __forceinline__ void store_chunk(__nv_bfloat16* c, int64_t ldc,
                                             const __nv_bfloat16* bias, int row, int col0, int cend,
                                             const uint32_t (&v)[32], bool vec_ok) {
@@ -98,6 +105,57 @@ __device__ __forceinline__ void store_chunk(__nv_bfloat16* c, int64_t ldc,
     for (int i = 0; i < 32; ++i)
       if (col0 + i < cend) dst[i] = __float2bfloat16_rn(f[i]);
   }
+}
+
+// The chain kernel's epilogue for one 32-row × 32-column chunk held one row
+// per lane (v = fp32 columns col0 .. col0 + 31 of row row0 + lane): round to
+// bf16 (+bias) and transpose through a 2 KB shared buffer (64-byte rows,
+// 16-byte chunks swizzled by row so that both the row-wise writes and the
+// column-wise reads touch each bank once per 128 bytes), then store with
+// each instruction covering 8 rows × 64 contiguous bytes instead of 32 rows
+// × 16 bytes.  Generic loads and stores only: no proxy fence, so nothing
+// waits for the SM's in-flight TMA or tensor-core traffic.
+__device__ __forceinline__ void emit_chunk(uint8_t* buf, const uint32_t (&v)[32],
+                                           __nv_bfloat16* c, int64_t ldc,
+                                           const __nv_bfloat16* bias, int row0, int Mr, int col0,
+                                           int cend, bool vec_ok, int lane) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float lo = __uint_as_float(v[2 * i]), hi = __uint_as_float(v[2 * i + 1]);
+    if (bias) {
+      const int cl = col0 + 2 * i;
+      if (cl < cend) lo += __bfloat162float(bias[cl]);
+      if (cl + 1 < cend) hi += __bfloat162float(bias[cl + 1]);
+    }
+    w[i] = pack_bf16x2(lo, hi);
+  }
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ sw) << 4)) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  __syncwarp();
+  const int q = lane & 3;
+  const int col = col0 + 8 * q;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int r = 8 * s + (lane >> 2);
+    const uint4 u = *reinterpret_cast<const uint4*>(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+    const int row = row0 + r;
+    if (row >= Mr || col >= cend) continue;
+    __nv_bfloat16* dst = c + static_cast<int64_t>(row) * ldc + col;
+    if (vec_ok && col + 8 <= cend) {
+      *reinterpret_cast<uint4*>(dst) = u;
+    } else {
+      const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (col + i < cend)
+          dst[i] = __ushort_as_bfloat16(static_cast<unsigned short>(e[i >> 1] >> (16 * (i & 1))));
+    }
+  }
+  __syncwarp();
 }
 
 constexpr int kGemmThreads = 6 * 32;
@@ -130,7 +188,7 @@ __device__ bool wait_rows_ready(const ChainArgs& g, int grp, int m_blk, int coun
   return true;
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kChainThreads, 1)
     umma_chain_kernel(const __grid_constant__ ChainMaps maps, const __grid_constant__ ChainArgs g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -156,7 +214,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1u);
-      mbar_init(&tempty[i], EPI_WARPS);
+      mbar_init(&tempty[i], C_EPI_WARPS);
     }
     mbar_init(fin, 1u);
     fence_mbar_init();
@@ -165,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == TMA_WARP && lane == 0 && blockIdx.x < g.total_tiles) {
+  if (warp == C_TMA_WARP && lane == 0 && blockIdx.x < g.total_tiles) {
     const ChainProblem& P = g.p[find_problem(g, blockIdx.x)];
     tma_prefetch_desc(&maps.m[P.map_a]);
     tma_prefetch_desc(&maps.m[P.map_b]);
@@ -181,7 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
   bool ok = true;
 
-  if (warp == TMA_WARP) {
+  if (warp == C_TMA_WARP) {
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -275,7 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-  } else if (warp == MMA_WARP) {
+  } else if (warp == C_MMA_WARP) {
     int s = 0;
     uint32_t ph = 0;
     int it = 0;
@@ -319,14 +377,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) umma_commit(&tfull[acc]);
       __syncwarp();
     }
-  } else if (warp < EPI_WARPS) {
+  } else if (warp < C_EPI_WARPS) {
     // Under programmatic dependent launch, write nothing before the previous
     // launch on the stream has finished (it may still read these buffers).
     griddep_wait();
     if (blockIdx.x == 0)  // the next launch's counter bank (the previous launch used it)
-      for (int i = threadIdx.x; i < g.n_counters; i += EPI_WARPS * 32) g.counters_next[i] = 0u;
+      for (int i = threadIdx.x; i < g.n_counters; i += C_EPI_WARPS * 32) g.counters_next[i] = 0u;
     int it = 0;
-    int epi_box = 0;  // boxes this warp has staged (rotating buffers)
     for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x, ++it) {
       const ChainProblem& P = g.p[find_problem(g, tile)];
       const int local = tile - P.tile_begin;
@@ -340,79 +397,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const bool vec_ok =
           ((reinterpret_cast<uintptr_t>(P.c) & 15u) == 0) && ((P.ldc & 7) == 0);
-      const int row0 = m_blk * BM + warp * 32;
-      const int row = row0 + lane;
+      const int quarter = warp & 3, half = warp >> 2;
+      const int row0 = m_blk * BM + quarter * 32;
       const int n0 = n_blk * P.bn;
       const int cend = min(P.Nc, n0 + P.bn);
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * MAX_BN);
-      const CUtensorMap* mc = P.map_c >= 0 ? &maps.m[P.map_c] : nullptr;
-      // One 32-column chunk: bf16 rounding (+bias) and the store.
-      auto emit = [&](const uint32_t (&v)[32], int c) {
-        const int col0 = n0 + c * 32;
-        if (mc) {
-          // Stage the warp's 32 × 32 box in shared memory (row = lane,
-          // 16-byte chunks swizzled so that the warp's writes hit every bank
-          // once per 128 bytes) and let TMA write it out with full-line
-          // stores; the map clips rows >= Mr and columns >= Nc.
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float lo = __uint_as_float(v[2 * i]), hi = __uint_as_float(v[2 * i + 1]);
-            if (P.bias) {
-              const int cl = col0 + 2 * i;
-              if (cl < cend) lo += __bfloat162float(P.bias[cl]);
-              if (cl + 1 < cend) hi += __bfloat162float(P.bias[cl + 1]);
-            }
-            w[i] = pack_bf16x2(lo, hi);
-          }
-          uint8_t* box = epi_stage + (warp * EPI_BOXES + (epi_box % EPI_BOXES)) * EPI_BOX;
-          if (epi_box >= EPI_BOXES) {
-            // The store that used this box last has read it.
-            if (lane == 0) bulk_wait_group_read<EPI_BOXES - 1>();
-            __syncwarp();
-          }
-          const int sw = (lane >> 1) & 3;
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ sw) << 4)) =
-                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(mc, box, col0, row0);
-            bulk_commit_group();
-          }
-          ++epi_box;
-        } else if (row < P.Mr) {
-          store_chunk(P.c, P.ldc, P.bias, row, col0, cend, v, vec_ok);
-        }
-      };
-      // Chunks alternate between two register sets: the TMEM load of chunk
-      // c + 1 is in flight while chunk c is rounded and stored.
+      uint8_t* bufs = epi_stage + warp * (2 * EPI_BOX);
+      // This warp's chunks are half, half + 2, ...  They alternate between
+      // two register sets (the TMEM load of the next chunk is in flight
+      // while one is rounded and stored) and two shared buffers.
       const int nch = (min(P.bn, cend - n0) + 31) / 32;
       uint32_t va[32], vb[32];
-      tmem_ld_32x32b_x32(t_row, va);
+      if (half < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(half * 32), va);
 #pragma unroll 1
-      for (int c = 0; c < nch; c += 2) {
+      for (int c = half; c < nch; c += 4) {
         tmem_ld_wait(va);
-        if (c + 1 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * 32), vb);
-        emit(va, c);
-        if (c + 1 < nch) {
+        if (c + 2 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * 32), vb);
+        emit_chunk(bufs, va, P.c, P.ldc, P.bias, row0, P.Mr, n0 + c * 32, cend, vec_ok, lane);
+        if (c + 2 < nch) {
           tmem_ld_wait(vb);
-          if (c + 2 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * 32), va);
-          emit(vb, c + 1);
+          if (c + 4 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 4) * 32), va);
+          emit_chunk(bufs + EPI_BOX, vb, P.c, P.ldc, P.bias, row0, P.Mr, n0 + (c + 2) * 32, cend,
+                     vec_ok, lane);
         }
       }
       tc_fence_before();
       if (P.signal_group >= 0) {
         // This warp's rows of the tile are written: make them visible to the
         // TMA loads of other CTAs, then count the arrival.
-        if (mc) {
-          if (lane == 0) bulk_wait_group<0>();
-        } else {
-          fence_proxy_async_global();
-        }
+        fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) {
           fence_proxy_async_global();
@@ -423,18 +437,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
-    // The staged boxes must stay in place until TMA has read them.
-    if (lane == 0) bulk_wait_group<0>();
-    __syncwarp();
   }
 
   // Teardown.  Every wait above is bounded, so every thread gets here.
-  if (warp == MMA_WARP && lane == 0) {
+  if (warp == C_MMA_WARP && lane == 0) {
     // All MMAs this thread issued are complete once fin flips.
     umma_commit(fin);
     mbar_wait_drain(fin, 0u, 2000000000ull);
   }
-  if (warp == TMA_WARP && lane == 0 && !ok) {
+  if (warp == C_TMA_WARP && lane == 0 && !ok) {
     // After a timeout: let any TMA load still in flight land before exit.
     for (int s = 0; s < STAGES; ++s)
       if (issued_phase[s] >= 0)
@@ -683,7 +694,7 @@ cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid,
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(std::max(1, grid));
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(kChainThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
