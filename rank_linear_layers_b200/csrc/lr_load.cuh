@@ -123,6 +123,24 @@ __device__ __forceinline__ uint2 shfl_down_u2(uint2 v, int d, int width) {
   return v;
 }
 
+// Bytes [sh, sh + 16) of the 32-byte window (lo, hi), sh even: the 8
+// elements that start sh bytes into the aligned granule lo.
+__device__ __forceinline__ uint4 window16(const uint4& lo, const uint4& hi, uint32_t sh) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t o[5];
+  switch (sh >> 2) {
+    case 0: o[0] = w[0]; o[1] = w[1]; o[2] = w[2]; o[3] = w[3]; o[4] = w[4]; break;
+    case 1: o[0] = w[1]; o[1] = w[2]; o[2] = w[3]; o[3] = w[4]; o[4] = w[5]; break;
+    case 2: o[0] = w[2]; o[1] = w[3]; o[2] = w[4]; o[3] = w[5]; o[4] = w[6]; break;
+    default: o[0] = w[3]; o[1] = w[4]; o[2] = w[5]; o[3] = w[6]; o[4] = w[7]; break;
+  }
+  if (sh & 2u) {
+    return make_uint4(__byte_perm(o[0], o[1], 0x5432), __byte_perm(o[1], o[2], 0x5432),
+                      __byte_perm(o[2], o[3], 0x5432), __byte_perm(o[3], o[4], 0x5432));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Zero the elements of an 8-element chunk whose index (0..7) is >= keep.
 __device__ __forceinline__ uint4 mask_tail8(uint4 v, int keep) {
   if (keep >= 8) return v;

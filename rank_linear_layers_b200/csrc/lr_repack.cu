@@ -12,6 +12,7 @@
 #include <algorithm>
 
 #include "lr_internal.h"
+#include "lr_load.cuh"
 
 namespace lr {
 
@@ -19,31 +20,6 @@ namespace {
 
 constexpr int kRepackThreads = 256;
 constexpr int kRepackU = 4;  // destination chunks in flight per thread
-
-__device__ __forceinline__ uint4 ld_nc16(uintptr_t a) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(a));
-  return v;
-}
-
-// Bytes [sh, sh + 16) of the 32-byte window (lo, hi), sh even.
-__device__ __forceinline__ uint4 window16(const uint4& lo, const uint4& hi, uint32_t sh) {
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t o[5];
-  switch (sh >> 2) {
-    case 0: o[0] = w[0]; o[1] = w[1]; o[2] = w[2]; o[3] = w[3]; o[4] = w[4]; break;
-    case 1: o[0] = w[1]; o[1] = w[2]; o[2] = w[3]; o[3] = w[4]; o[4] = w[5]; break;
-    case 2: o[0] = w[2]; o[1] = w[3]; o[2] = w[4]; o[3] = w[5]; o[4] = w[6]; break;
-    default: o[0] = w[3]; o[1] = w[4]; o[2] = w[5]; o[3] = w[6]; o[4] = w[7]; break;
-  }
-  if (sh & 2u) {
-    return make_uint4(__byte_perm(o[0], o[1], 0x5432), __byte_perm(o[1], o[2], 0x5432),
-                      __byte_perm(o[2], o[3], 0x5432), __byte_perm(o[3], o[4], 0x5432));
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
 
 // One thread per 16-byte destination chunk (row k, elements 8j .. 8j+7):
 // the chunk's source bytes span at most two aligned 16-byte granules of the
@@ -68,8 +44,8 @@ __global__ void __launch_bounds__(kRepackThreads) repack_chunks_kernel(
         const uintptr_t p = reinterpret_cast<uintptr_t>(src + static_cast<int64_t>(k) * lds + 8 * j);
         const uintptr_t a = p & ~static_cast<uintptr_t>(15);
         shift[u] = static_cast<uint32_t>(p & 15u);
-        lo[u] = ld_nc16(a);
-        hi2[u] = (shift[u] != 0u && a + 16 < hi) ? ld_nc16(a + 16) : make_uint4(0, 0, 0, 0);
+        lo[u] = ld_nc_v4(a);
+        hi2[u] = (shift[u] != 0u && a + 16 < hi) ? ld_nc_v4(a + 16) : make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
@@ -79,13 +55,7 @@ __global__ void __launch_bounds__(kRepackThreads) repack_chunks_kernel(
         const uint32_t k = q / cpr, j = q - k * cpr;
         uint4 v = window16(lo[u], hi2[u], shift[u]);
         const int valid = static_cast<int>(cols) - static_cast<int>(8 * j);
-        if (valid < 8) {
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (e >= valid) w[e >> 1] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-          v = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        if (valid < 8) v = mask_tail8(v, valid);
         *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(k) * ldd + 8 * j) = v;
       }
     }
