@@ -614,6 +614,142 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
 }
 
 
+// The projections of a group at prefill sizes, in one chain launch.
+// Projections that share X (same pointer and K) form a set: their A factors
+// are copied side by side into one [K, Σ r_i] factor (each r_i rounded up to
+// 8 columns, so every slice starts on a 16-byte boundary) and the set runs
+// one GEMM1 T_set = X·A_set; projection i then runs GEMM2 Y_i = T_set[:,
+// off_i : off_i + r_i]·B_i (+bias_i), waiting for T_set's row blocks.  Its
+// K loop may read T_set columns past r_i (the next slice) but B_i's rows
+// past r_i read as zero, so those products are zero.  X is read once per set
+// and the whole layer is one launch.  Returns LR_ERR_UNSUPPORTED (before any
+// launch) when the group does not fit one launch's tables.
+lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* projs, int n,
+                            int64_t M) {
+  struct Set {
+    const void* X;
+    int64_t K;
+    std::vector<int> members;
+    int64_t width = 0;  // columns of T_set (sum of slices)
+    bool concat = false;  // A copied into a concatenated factor
+  };
+  std::vector<Set> sets;
+  std::vector<int64_t> off(static_cast<size_t>(n), 0);
+  std::vector<int> set_of(static_cast<size_t>(n), -1);
+  int gemm2 = 0;
+  for (int i = 0; i < n; ++i) {
+    const lr_proj& p = projs[i];
+    if (p.N == 0 || p.K == 0 || p.r == 0) continue;
+    int si = -1;
+    for (size_t k = 0; k < sets.size(); ++k)
+      if (sets[k].X == p.X && sets[k].K == p.K) si = static_cast<int>(k);
+    if (si < 0) {
+      sets.push_back(Set{p.X, p.K, {}, 0, false});
+      si = static_cast<int>(sets.size()) - 1;
+    }
+    Set& st = sets[static_cast<size_t>(si)];
+    off[static_cast<size_t>(i)] = st.width;
+    st.width += static_cast<int64_t>(align_up(static_cast<size_t>(p.r), 8));
+    st.members.push_back(i);
+    set_of[static_cast<size_t>(i)] = si;
+    ++gemm2;
+  }
+  if (static_cast<int>(sets.size()) + gemm2 > kChainMaxProbs ||
+      3 * static_cast<int>(sets.size()) + gemm2 > kChainMaxMaps)
+    return LR_ERR_UNSUPPORTED;
+  // Workspace: T per set, concatenated factors, realigned X and B copies.
+  size_t need = 0;
+  for (Set& st : sets) {
+    const lr_proj& p0 = projs[st.members[0]];
+    st.concat = st.members.size() > 1 || !tma_ok(p0.A, p0.r);
+    need += align_up(static_cast<size_t>(M) * st.width * 2, 256);
+    if (st.concat) need += align_up(static_cast<size_t>(st.K) * st.width * 2, 256);
+    need += repack_bytes(st.X, st.K, M, st.K);
+  }
+  for (int i = 0; i < n; ++i)
+    if (set_of[static_cast<size_t>(i)] >= 0) need += repack_bytes(projs[i].B, projs[i].N, projs[i].r, projs[i].N);
+  char *zero = nullptr, *scratch = nullptr;
+  lr_status stt = workspace(stream, 0, need, &zero, &scratch);
+  if (stt != LR_OK) return stt;
+  // Empty contractions: Y = bias.
+  for (int i = 0; i < n; ++i) {
+    const lr_proj& p = projs[i];
+    if (M > 0 && p.N > 0 && (p.K == 0 || p.r == 0)) {
+      stt = launched(launch_fill_bias(static_cast<__nv_bfloat16*>(p.Y), p.ld_y, M, p.N,
+                                      static_cast<const __nv_bfloat16*>(p.bias), stream));
+      if (stt != LR_OK) return stt;
+    }
+  }
+  // Copies (repack kernels), then the chain launch.
+  int repacks = 0;
+  struct SetOps {
+    void* T;
+    Operand x, a;
+  };
+  std::vector<SetOps> ops(sets.size());
+  for (size_t k = 0; k < sets.size(); ++k) {
+    Set& st = sets[k];
+    ops[k].T = scratch;
+    scratch += align_up(static_cast<size_t>(M) * st.width * 2, 256);
+    stt = tma_operand(d, stream, st.X, st.K, M, st.K, &scratch, &ops[k].x, &repacks);
+    if (stt != LR_OK) return stt;
+    if (st.concat) {
+      __nv_bfloat16* cat = reinterpret_cast<__nv_bfloat16*>(scratch);
+      scratch += align_up(static_cast<size_t>(st.K) * st.width * 2, 256);
+      for (int i : st.members) {
+        const lr_proj& p = projs[i];
+        stt = launched(launch_repack(static_cast<const __nv_bfloat16*>(p.A), p.r,
+                                     span_bytes(p.K, p.r, p.r), cat + off[static_cast<size_t>(i)],
+                                     st.width, p.K, p.r, d->sms, stream, repacks > 0));
+        if (stt != LR_OK) return stt;
+        ++repacks;
+      }
+      ops[k].a = Operand{cat, st.width};
+    } else {
+      const lr_proj& p = projs[st.members[0]];
+      ops[k].a = Operand{p.A, p.r};
+    }
+  }
+  std::vector<Operand> bops(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    if (set_of[static_cast<size_t>(i)] < 0) continue;
+    const lr_proj& p = projs[i];
+    stt = tma_operand(d, stream, p.B, p.N, p.r, p.N, &scratch, &bops[static_cast<size_t>(i)], &repacks);
+    if (stt != LR_OK) return stt;
+  }
+  const bool after_repack = repacks > 0;
+  auto dep = [&](const void* used, const void* given) { return !after_repack || used != given; };
+  ChainBuild cb;
+  std::vector<int> tmap(sets.size());
+  for (size_t k = 0; k < sets.size(); ++k) {
+    const Set& st = sets[k];
+    const lr_proj& p0 = projs[st.members[0]];
+    const int64_t nc = st.concat ? st.width : p0.r;  // T columns GEMM1 writes
+    int mx, ma, mt;
+    if ((stt = chain_map(cb, ops[k].x.p, st.K, M, ops[k].x.ld, true, &mx)) != LR_OK) return stt;
+    if ((stt = chain_map(cb, ops[k].a.p, nc, st.K, ops[k].a.ld, false, &ma)) != LR_OK) return stt;
+    // T's columns past nc are never written: the map ends there (they read as
+    // zero); a concatenated T's slice pads are written as zero by GEMM1.
+    if ((stt = chain_map(cb, ops[k].T, nc, M, st.width, true, &mt)) != LR_OK) return stt;
+    tmap[k] = mt;
+    stt = chain_problem(cb, mx, 0, ma, M, nc, st.K, ops[k].T, st.width, nullptr, -1,
+                        static_cast<int>(k), dep(ops[k].x.p, st.X), dep(ops[k].a.p, p0.A));
+    if (stt != LR_OK) return stt;
+  }
+  for (size_t k = 0; k < sets.size(); ++k) {
+    for (int i : sets[k].members) {
+      const lr_proj& p = projs[i];
+      const Operand& b = bops[static_cast<size_t>(i)];
+      int mb;
+      if ((stt = chain_map(cb, b.p, p.N, p.r, b.ld, false, &mb)) != LR_OK) return stt;
+      stt = chain_problem(cb, tmap[k], static_cast<int>(off[static_cast<size_t>(i)]), mb, M, p.N,
+                          p.r, p.Y, p.ld_y, p.bias, static_cast<int>(k), -1, false, dep(b.p, p.B));
+      if (stt != LR_OK) return stt;
+    }
+  }
+  return run_chain(d, stream, cb);
+}
+
 // Two projections' outputs may interleave (gate and up writing the two halves
 // of one packed buffer) but must not share an element.  Conservative: equal
 // row strides and no row that spills into the next are required when the byte
@@ -686,6 +822,16 @@ lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* str
           return LR_ERR_INVALID_ARG;
       }
     }
+  }
+  // Prefill sizes: the whole group in one chain launch (see run_group_prefill).
+  const int path = g_path.load();
+  if (M > 16 && path != 1 && path != 4 && n_proj > 0) {
+    DeviceInfo* d = nullptr;
+    int dev = 0;
+    lr_status st = device_info(&d, &dev);
+    if (st != LR_OK) return st;
+    st = run_group_prefill(d, static_cast<cudaStream_t>(stream), projs, n_proj, M);
+    if (st != LR_ERR_UNSUPPORTED) return st;
   }
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];

@@ -12,7 +12,7 @@ import pytest
 
 import lrgen
 import oracle
-from helpers import compare, to_dev, to_f64
+from helpers import compare, compare_prefill, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -60,3 +60,51 @@ def test_decoder_layer_group(M, n_int):
             assert np.array_equal(Y1, outs[n]), f"group vs single differ for {n}"
         else:
             compare(outs[n], Y1, f"group vs single {n}")
+
+
+def _group_case(specs, M, seed):
+    """specs: list of (x_name, K, r, N, bias).  Returns inputs, entries, outputs."""
+    import torch
+    import rank_linear_layers_b200 as lr
+    xs, entries, outs, probs = {}, [], [], []
+    for i, (xn, K, r, N, bias) in enumerate(specs):
+        p = lrgen.lowrank_problem(M, K, r, N, seed=seed + i, bias=bias)
+        if xn not in xs:
+            xs[xn] = (p["X"], to_dev(p["X"]))
+        p["X"] = xs[xn][0]
+        Y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+        e = dict(X=xs[xn][1], A=to_dev(p["A"]), B=to_dev(p["B"]), K=K, r=r, N=N, Y=Y)
+        if bias:
+            e["bias"] = to_dev(p["bias"])
+        entries.append(e)
+        outs.append(Y)
+        probs.append(p)
+    lr.lr_linear_group(entries, M)
+    torch.cuda.synchronize()
+    assert lr.last_device_status() == lr.LR_OK
+    return entries, outs, probs
+
+
+@pytest.mark.parametrize("M", [17, 300])
+def test_group_sets_share_x(M):
+    """Sets of projections sharing X (concatenated factors, one GEMM1 per set,
+    one launch), odd ranks and K, a misaligned X, bias on some: every output
+    equals the oracle, and bit for bit the projection run alone."""
+    import rank_linear_layers_b200 as lr
+    specs = [("x1", 136, 37, 100, False), ("x1", 136, 64, 64, False), ("x1", 136, 5, 517, True),
+             ("x2", 333, 257, 40, True), ("x2", 333, 1, 8, False), ("x3", 64, 7, 9, False),
+             ("x4", 256, 128, 256, False)]
+    entries, outs, probs = _group_case(specs, M, seed=40)
+    for e, Y, p in zip(entries, outs, probs):
+        compare_prefill(to_f64(Y), p, what=f"group K={p['K']} r={p['r']} N={p['N']}")
+        Y1 = lr.lr_linear(e["X"], e["A"], e["B"], e.get("bias"))
+        assert np.array_equal(to_f64(Y1), to_f64(Y)), f"group vs single r={p['r']}"
+
+
+def test_group_larger_than_one_launch():
+    """More projections than one launch's tables hold: run one by one."""
+    specs = [(f"x{i % 3}", 96, 9 + i, 40 + i, i % 2 == 0) for i in range(14)]
+    entries, outs, probs = _group_case(specs, 64, seed=70)
+    for Y, p in zip(outs, probs):
+        compare(to_f64(Y), oracle.lr_linear(p["X"], p["A"], p["B"], p.get("bias")),
+                f"group(14) r={p['r']}")
