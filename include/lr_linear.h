@@ -171,11 +171,17 @@ int lr_last_cuda_error(void);
  *   the width that spreads the launch's tiles most evenly over the SMs);
  *   32..256 in steps of 32 forces that width for every GEMM (for tests and
  *   tuning).  Other values return LR_ERR_INVALID_ARG.
- * All three are process-wide and take effect on the next call.
+ * lr_set_split_k — on = 1 (the default): a prefill GEMM with fewer tiles
+ *   than half the SMs and at least 16 k blocks of 64 (GEMM1 at small ranks)
+ *   splits its K loop over several CTAs, which add fp32 partial sums into a
+ *   workspace; the last one rounds and stores.  on = 0 turns it off (for
+ *   tests and tuning); other values return LR_ERR_INVALID_ARG.
+ * All four are process-wide and take effect on the next call.
  */
 lr_status lr_set_path(int path);
 lr_status lr_set_wait_limit_ns(int64_t ns);
 lr_status lr_set_tile_n(int bn);
+lr_status lr_set_split_k(int on);
 
 /*
  * lr_set_withhold_first_stage — testing failure detection only.  With on = 1,

@@ -32,7 +32,7 @@ EXPORTS = (
     "lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense", "lr_last_device_status",
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
     "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
-    "lr_set_withhold_first_stage", "lr_set_tile_n",
+    "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k",
 )
 
 
@@ -78,6 +78,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_set_wait_limit_ns.argtypes = [i64]
     L.lr_set_withhold_first_stage.argtypes = [ctypes.c_int]
     L.lr_set_tile_n.argtypes = [ctypes.c_int]
+    L.lr_set_split_k.argtypes = [ctypes.c_int]
     L.lr_kernel_launch_count.argtypes = []
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
@@ -85,7 +86,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
                  "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces", "lr_set_withhold_first_stage",
-                 "lr_set_tile_n"):
+                 "lr_set_tile_n", "lr_set_split_k"):
         getattr(L, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = L
@@ -215,6 +216,11 @@ def set_wait_limit_ns(ns: int):
 def set_tile_n(bn: int):
     """Force the prefill tile width (32..256, multiple of 32); 0 = automatic."""
     _check(lib().lr_set_tile_n(bn), "lr_set_tile_n")
+
+
+def set_split_k(on: bool):
+    """Split long K loops of small prefill GEMMs over several CTAs (default on)."""
+    _check(lib().lr_set_split_k(1 if on else 0), "lr_set_split_k")
 
 
 def set_withhold_first_stage(on: bool):

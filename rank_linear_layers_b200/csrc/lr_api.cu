@@ -25,6 +25,7 @@ std::atomic<long long> g_wait_ns{0};
 std::atomic<long long> g_launches{0};
 std::atomic<int> g_withhold{0};
 std::atomic<int> g_tile_n{0};
+std::atomic<int> g_split_k{1};
 constexpr long long kDefaultWaitNs = 2000000000LL;
 
 struct DeviceInfo {
@@ -45,6 +46,9 @@ struct Workspace {
   unsigned int* ctrs = nullptr;
   size_t n_ctrs = 0;
   unsigned int launches = 0;
+  // Split-K partial sums of the chain kernel (fp32, zero at rest).
+  float* split_ws = nullptr;
+  size_t split_cap = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
@@ -309,6 +313,28 @@ lr_status chain_counters(cudaStream_t stream, size_t n, unsigned int** bank,
   return LR_OK;
 }
 
+// fp32 split-K workspace of `bytes` on `stream`, zero at rest.
+lr_status chain_split_ws(cudaStream_t stream, size_t bytes, float** out) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  if (bytes > w.split_cap) {
+    if (w.split_ws) {
+      LR_CUDA(cudaStreamSynchronize(stream));
+      LR_CUDA(cudaFree(w.split_ws));
+      w.split_ws = nullptr;
+      w.split_cap = 0;
+    }
+    const size_t cap = align_up(bytes + bytes / 4, 1 << 20);
+    LR_CUDA(cudaMalloc(&w.split_ws, cap));
+    LR_CUDA(cudaMemsetAsync(w.split_ws, 0, cap, stream));
+    w.split_cap = cap;
+  }
+  *out = w.split_ws;
+  return LR_OK;
+}
+
 // One launch of the chain kernel under construction.
 struct ChainBuild {
   ChainMaps maps{};
@@ -468,15 +494,46 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
   int groups = 0, stride = 1;
   for (int i = 0; i < a.n_prob; ++i) {
     ChainProblem& P = a.p[i];
+    if (P.signal_group >= 0) groups = std::max(groups, P.signal_group + 1);
+  }
+  // Split K for a GEMM with too few tiles to fill half the SMs and a long
+  // K loop (GEMM1 at small ranks): up to one split per 8 k blocks, as many
+  // as fill the SMs.
+  int64_t split_floats = 0;
+  for (int i = 0; i < a.n_prob; ++i) {
+    ChainProblem& P = a.p[i];
     P.bn = bn[i];
     P.tiles_m = static_cast<int>(ceil_div(P.Mr, kGemmBM));
     P.tiles_n = static_cast<int>(ceil_div(P.Nc, P.bn));
+    const int64_t tiles = static_cast<int64_t>(P.tiles_m) * P.tiles_n;
+    const int nkb = static_cast<int>(ceil_div(P.Kc, kGemmBK));
+    int splits = 1;
+    if (g_split_k.load() && tiles * 2 <= d->sms && nkb >= 16)
+      splits = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({nkb / 8, d->sms / tiles, 16})));
+    P.kb_per_split = static_cast<int>(ceil_div(nkb, splits));
+    P.splits = static_cast<int>(ceil_div(nkb, P.kb_per_split));
+    P.split_group = -1;
+    if (P.splits > 1) {
+      P.split_group = groups++;
+      stride = static_cast<int>(std::max<int64_t>(stride, tiles * kChainEpiWarps));
+      P.ws_ld = static_cast<int64_t>(P.tiles_n) * P.bn;
+      split_floats += static_cast<int64_t>(P.tiles_m) * kGemmBM * P.ws_ld;
+    }
     P.tile_begin = static_cast<int>(total);
-    total += static_cast<int64_t>(P.tiles_m) * P.tiles_n;
+    total += tiles * P.splits;
     if (total > kMaxDim) return LR_ERR_UNSUPPORTED;
-    if (P.signal_group >= 0) {
-      groups = std::max(groups, P.signal_group + 1);
-      stride = std::max(stride, P.tiles_m);
+    if (P.signal_group >= 0) stride = std::max(stride, P.tiles_m);
+  }
+  if (split_floats > 0) {
+    float* ws = nullptr;
+    lr_status st = chain_split_ws(stream, static_cast<size_t>(split_floats) * 4, &ws);
+    if (st != LR_OK) return st;
+    for (int i = 0; i < a.n_prob; ++i) {
+      ChainProblem& P = a.p[i];
+      if (P.splits > 1) {
+        P.ws = ws;
+        ws += static_cast<int64_t>(P.tiles_m) * kGemmBM * P.ws_ld;
+      }
     }
   }
   for (int i = 0; i < a.n_prob; ++i) {
@@ -953,6 +1010,17 @@ lr_status lr_last_device_status(void* stream) {
   h.code |= static_code;
   if (h.code == 0 && h.abort == 0) return LR_OK;
   LR_CUDA(cudaMemset(d->status, 0, sizeof(DevStatus)));
+  {
+    // A launch that gave up may have left partial sums behind: zero what
+    // this stream's workspace must hold zero between calls.
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_ws.find({dev, static_cast<cudaStream_t>(stream)});
+    if (it != g_ws.end()) {
+      if (it->second.ptr && it->second.zero_bytes)
+        LR_CUDA(cudaMemset(it->second.ptr, 0, it->second.zero_bytes));
+      if (it->second.split_ws) LR_CUDA(cudaMemset(it->second.split_ws, 0, it->second.split_cap));
+    }
+  }
   return (h.code & LR_DEV_TIMEOUT) ? LR_ERR_TIMEOUT : LR_ERR_CUDA;
 }
 
@@ -984,6 +1052,12 @@ lr_status lr_set_wait_limit_ns(int64_t ns) {
 
 int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
 
+lr_status lr_set_split_k(int on) {
+  if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
+  g_split_k.store(on);
+  return LR_OK;
+}
+
 lr_status lr_set_tile_n(int bn) {
   if (bn < 0 || bn > 256 || bn % 32 != 0) return LR_ERR_INVALID_ARG;
   g_tile_n.store(bn);
@@ -1001,11 +1075,12 @@ lr_status lr_release_workspaces(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_ws) {
-    if (!kv.second.ptr && !kv.second.ctrs) continue;
+    if (!kv.second.ptr && !kv.second.ctrs && !kv.second.split_ws) continue;
     cudaSetDevice(kv.first.first);
     cudaStreamSynchronize(kv.first.second);
     if (kv.second.ptr) cudaFree(kv.second.ptr);
     if (kv.second.ctrs) cudaFree(kv.second.ctrs);
+    if (kv.second.split_ws) cudaFree(kv.second.split_ws);
   }
   g_ws.clear();
   for (auto& kv : g_stage) {

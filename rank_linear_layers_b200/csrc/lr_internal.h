@@ -141,6 +141,14 @@ struct ChainProblem {
   int wait_count;    // arrivals that complete one row block of that group
   int signal_group;  // -1, or the counter group this problem arrives on
   int dep_a, dep_b;  // operand written by the previous launch on the stream
+  // Split K: each output tile is `splits` tiles of the launch, each over
+  // kb_per_split k blocks; partial sums are added (fp32 vector reductions)
+  // into ws [tiles_m·128, ws_ld], zero at rest, and the last split to
+  // finish a warp's region (arrival counter in group split_group, one per
+  // tile and epilogue warp) rounds, stores and re-zeroes it.
+  int splits, kb_per_split, split_group;
+  float* ws;
+  int64_t ws_ld;
 };
 
 struct ChainArgs {

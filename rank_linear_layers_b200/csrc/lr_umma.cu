@@ -158,6 +158,29 @@ __device__ __forceinline__ void emit_chunk(uint8_t* buf, const uint32_t (&v)[32]
   __syncwarp();
 }
 
+// Split K: add one 32-row × 32-column fp32 chunk (one row per lane, as read
+// from TMEM) into the workspace, transposed through the warp's 4 KB buffer
+// (128-byte rows, 16-byte chunks swizzled by row) so that each vector
+// reduction covers 4 rows × 128 contiguous bytes.
+__device__ __forceinline__ void split_add_chunk(uint8_t* buf, const uint32_t (&v)[32], float* ws,
+                                                int64_t ld, int row0, int col0, int lane) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int c = lane & 7;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int r = 4 * s + (lane >> 3);
+    const uint4 u = *reinterpret_cast<const uint4*>(buf + r * 128 + ((c ^ (r & 7)) << 4));
+    float4* dst = reinterpret_cast<float4*>(ws + static_cast<int64_t>(row0 + r) * ld + col0 + 4 * c);
+    atomicAdd(dst, make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                               __uint_as_float(u.w)));
+  }
+  __syncwarp();
+}
+
 constexpr int kGemmThreads = 6 * 32;
 
 __device__ __forceinline__ int find_problem(const ChainArgs& g, int tile) {
@@ -247,18 +270,20 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x) {
         const ChainProblem& P = g.p[find_problem(g, tile)];
         const int local = tile - P.tile_begin;
-        const int m_blk = local / P.tiles_n, n_blk = local - m_blk * P.tiles_n;
-        const int num_kb = (P.Kc + BK - 1) / BK;
+        const int otile = local / P.splits, kbase = (local - otile * P.splits) * P.kb_per_split;
+        const int m_blk = otile / P.tiles_n, n_blk = otile - m_blk * P.tiles_n;
+        const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
         const int nbox = (P.bn + 63) / 64;
         const uint32_t bytes = A_STAGE + nbox * B_ATOM;
         const CUtensorMap* ma = &maps.m[P.map_a];
         const CUtensorMap* mb = &maps.m[P.map_b];
         auto load_a = [&](int st, int kb) {
-          tma_load_2d(stage_a(st), ma, &full[st], P.a_col0 + kb * BK, m_blk * BM);
+          tma_load_2d(stage_a(st), ma, &full[st], P.a_col0 + (kbase + kb) * BK, m_blk * BM);
         };
         auto load_b = [&](int st, int kb) {
           for (int c = 0; c < nbox; ++c)
-            tma_load_2d(stage_b(st) + c * B_ATOM, mb, &full[st], n_blk * P.bn + c * 64, kb * BK);
+            tma_load_2d(stage_b(st) + c * B_ATOM, mb, &full[st], n_blk * P.bn + c * 64,
+                        (kbase + kb) * BK);
         };
         const bool gated_a = P.dep_a || P.wait_group >= 0;
         const bool gated_b = P.dep_b;
@@ -339,7 +364,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x, ++it) {
       const ChainProblem& P = g.p[find_problem(g, tile)];
-      const int num_kb = (P.Kc + BK - 1) / BK;
+      const int local = tile - P.tile_begin;
+      const int kbase = (local - (local / P.splits) * P.splits) * P.kb_per_split;
+      const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
       const uint32_t idesc = idesc_bf16_f32(BM, P.bn, false, true);
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
@@ -356,7 +383,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         }
         tc_fence_after();
         if (lane == 0) {
-          const int krem = P.Kc - kb * BK;
+          const int krem = P.Kc - (kbase + kb) * BK;
           const int nk = krem >= BK ? BK / 16 : (krem + 15) / 16;
           const uint32_t a0 = smem_u32(stage_a(s));
           const uint32_t b0 = smem_u32(stage_b(s));
@@ -387,7 +414,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     for (int tile = blockIdx.x; tile < g.total_tiles && ok; tile += gridDim.x, ++it) {
       const ChainProblem& P = g.p[find_problem(g, tile)];
       const int local = tile - P.tile_begin;
-      const int m_blk = local / P.tiles_n, n_blk = local - m_blk * P.tiles_n;
+      const int otile = local / P.splits;
+      const int m_blk = otile / P.tiles_n, n_blk = otile - m_blk * P.tiles_n;
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
       if (!mbar_wait(&tfull[acc], aph, g.wait, kWhereEpilogue)) {
@@ -409,21 +437,60 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       // while one is rounded and stored) and two shared buffers.
       const int nch = (min(P.bn, cend - n0) + 31) / 32;
       uint32_t va[32], vb[32];
-      if (half < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(half * 32), va);
+      bool last = true;  // this warp's region of the output tile is final
+      if (P.splits == 1) {
+        if (half < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(half * 32), va);
 #pragma unroll 1
-      for (int c = half; c < nch; c += 4) {
-        tmem_ld_wait(va);
-        if (c + 2 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * 32), vb);
-        emit_chunk(bufs, va, P.c, P.ldc, P.bias, row0, P.Mr, n0 + c * 32, cend, vec_ok, lane);
-        if (c + 2 < nch) {
-          tmem_ld_wait(vb);
-          if (c + 4 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 4) * 32), va);
-          emit_chunk(bufs + EPI_BOX, vb, P.c, P.ldc, P.bias, row0, P.Mr, n0 + (c + 2) * 32, cend,
-                     vec_ok, lane);
+        for (int c = half; c < nch; c += 4) {
+          tmem_ld_wait(va);
+          if (c + 2 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 2) * 32), vb);
+          emit_chunk(bufs, va, P.c, P.ldc, P.bias, row0, P.Mr, n0 + c * 32, cend, vec_ok, lane);
+          if (c + 2 < nch) {
+            tmem_ld_wait(vb);
+            if (c + 4 < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 4) * 32), va);
+            emit_chunk(bufs + EPI_BOX, vb, P.c, P.ldc, P.bias, row0, P.Mr, n0 + (c + 2) * 32,
+                       cend, vec_ok, lane);
+          }
+        }
+      } else {
+        // Split K: add this split's partial sums into the workspace; the
+        // last split of this warp's region rounds, stores and re-zeroes it.
+#pragma unroll 1
+        for (int c = half; c < nch; c += 2) {
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), va);
+          tmem_ld_wait(va);
+          split_add_chunk(bufs, va, P.ws, P.ws_ld, row0, n0 + c * 32, lane);
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned int before = 0;
+        if (lane == 0)
+          before = atomicAdd(g.counters + static_cast<int64_t>(P.split_group) * g.ctr_stride +
+                                 static_cast<int64_t>(otile) * C_EPI_WARPS + warp,
+                             1u);
+        before = __shfl_sync(0xffffffffu, before, 0);
+        last = (before == static_cast<unsigned int>(P.splits - 1));
+        if (last) {
+          __threadfence();
+#pragma unroll 1
+          for (int c = half; c < nch; c += 2) {
+            float4* src = reinterpret_cast<float4*>(
+                P.ws + static_cast<int64_t>(row0 + lane) * P.ws_ld + n0 + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 f = __ldcg(src + q);
+              va[4 * q] = __float_as_uint(f.x);
+              va[4 * q + 1] = __float_as_uint(f.y);
+              va[4 * q + 2] = __float_as_uint(f.z);
+              va[4 * q + 3] = __float_as_uint(f.w);
+              __stcg(src + q, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+            emit_chunk(bufs, va, P.c, P.ldc, P.bias, row0, P.Mr, n0 + c * 32, cend, vec_ok, lane);
+          }
         }
       }
       tc_fence_before();
-      if (P.signal_group >= 0) {
+      if (P.signal_group >= 0 && last) {
         // This warp's rows of the tile are written: make them visible to the
         // TMA loads of other CTAs, then count the arrival.
         fence_proxy_async_global();

@@ -60,8 +60,10 @@ def compare_prefill(Y, p, rows=None, what=""):
     passes only if (a) the same arithmetic done on the CPU — fp32 products,
     T rounded to bf16, fp32 second contraction, bias, Y rounded to bf16 —
     fails the bar too, by at least as much, and (b) the GPU output agrees
-    with that CPU result to within 2 bf16 ulps element by element (the two
-    accumulate in different orders).  A wrong kernel fails (b)."""
+    with that CPU result element by element within what the two computations
+    may legitimately differ by: one bf16 rounding of Y (2^-7·|Y|) plus one
+    bf16 rounding step of each element of T, whose fp32 sums are formed in
+    different orders (2^-8·(|T|·|B|)).  A wrong kernel fails (b)."""
     import oracle
     Yref = oracle.lr_linear(p["X"], p["A"], p["B"], p.get("bias"), rows=rows)
     try:
@@ -76,12 +78,13 @@ def compare_prefill(Y, p, rows=None, what=""):
         if p.get("bias") is not None:
             Z = Z + lrgen.bf16_to_f64(p["bias"])
         E = _bf16_round(Z)
+        S = np.abs(T) @ np.abs(B)
         rms = float(np.sqrt(np.mean(Yref ** 2)))
         e_gpu = float(np.abs(np.asarray(Y) - Yref).max()) / rms
         e_cpu = float(np.abs(E - Yref).max()) / rms
         assert e_cpu > MAX_ERR_RMS and e_gpu <= e_cpu * 1.05, \
             f"{what}: GPU max|err| {e_gpu:.3e}·RMS, same roundings on the CPU {e_cpu:.3e}·RMS"
-        ulp = np.maximum(np.abs(E), 1e-30) * 2.0 ** -7
-        assert np.all(np.abs(np.asarray(Y) - E) <= 2 * ulp + 1e-30), \
-            f"{what}: GPU differs from the CPU rounding model by more than 2 bf16 ulps"
+        allowed = 2.0 ** -7 * np.abs(E) + 2.0 ** -8 * S
+        assert np.all(np.abs(np.asarray(Y) - E) <= allowed), \
+            f"{what}: GPU differs from the CPU rounding model beyond one rounding of Y and of T"
         return e_gpu, None

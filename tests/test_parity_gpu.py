@@ -126,6 +126,52 @@ def test_prefill_tile_plan_around_1024(lr, r):
     compare(Y[rows], ref(p, rows=rows), f"r={r} sampled rows")
 
 
+@pytest.mark.parametrize("M,K,r,N", [
+    (300, 2048, 37, 300),     # 3 GEMM1 tiles, 32 k blocks: split 4 ways
+    (129, 1000, 8, 77),       # ragged M, K not a multiple of 64
+    (640, 4096, 64, 1000),
+])
+def test_prefill_split_k(lr, M, K, r, N):
+    """GEMM1 with too few tiles splits its K loop over CTAs (fp32 partial
+    sums, the last split rounds T); the same with splitting turned off."""
+    p = lrgen.lowrank_problem(M, K, r, N, seed=K + r, bias=True)
+    Yr = ref(p)
+    Ys = run_gpu(lr, p, lr.PATH_PREFILL)
+    lr.set_split_k(False)
+    try:
+        Y1 = run_gpu(lr, p, lr.PATH_PREFILL)
+    finally:
+        lr.set_split_k(True)
+    compare(Ys, Yr, f"split-K {M}x{K}x{r}x{N}")
+    compare(Y1, Yr, f"no split {M}x{K}x{r}x{N}")
+    # Repeated calls: the split workspace must be zero again after each.
+    for _ in range(2):
+        compare(run_gpu(lr, p, lr.PATH_PREFILL), Yr, "split-K repeated")
+
+
+def test_sweep_small_ranks_sampled_rows(lr):
+    """M = K = N = 4096 at r = 64 and 128 (the small-rank end of the sweep)."""
+    for r in (64, 128):
+        p = lrgen.lowrank_problem(4096, 4096, r, 4096, seed=r)
+        Y = run_gpu(lr, p)
+        rows = np.concatenate([np.random.default_rng(r).choice(4096, 40, replace=False), [0, 4095]])
+        compare(Y[rows], ref(p, rows=rows), f"r={r} sampled rows")
+
+
+def test_dense_split_k(lr):
+    """lr_dense with a long K and few tiles (split K), bias, ragged N."""
+    import torch
+    M, K, N = 256, 8192, 70
+    p = lrgen.lowrank_problem(M, K, N, 1, seed=5, bias=False)
+    bias = lrgen.lowrank_problem(1, 1, 1, N, seed=6, bias=True)["bias"]
+    X, W = to_dev(p["X"]), to_dev(p["A"])
+    Y = lr.lr_dense(X, W, to_dev(bias))
+    torch.cuda.synchronize()
+    eye = np.zeros((N, N), dtype=np.uint16)
+    eye[np.arange(N), np.arange(N)] = 0x3F80  # bf16 1.0: X·W·I through the oracle
+    compare(to_f64(Y), oracle.lr_linear(p["X"], p["A"], eye, bias), "dense split-K")
+
+
 def test_decode_and_prefill_agree_at_m16(lr):
     p = lrgen.lowrank_problem(16, 512, 300, 640, seed=3, bias=True)
     Yd = run_gpu(lr, p, lr.PATH_DECODE)
