@@ -439,15 +439,17 @@ def run_ours(args):
     value, t_max = aggregate(fl_step * args.steps, t, world)
     ms = t_max / args.steps * 1e3
 
-    # Roofline of the prefill kernels: two launches of the tcgen05 GEMM per
-    # step (T = X·A, then Y = T·B), each doing half of the step's FLOPs.
+    # Roofline of the prefill step: one launch of the tcgen05 chain kernel
+    # (GEMM1 T = X·A and GEMM2 Y = T·B, all of the step's FLOPs), after one
+    # repack launch for A (r = 1741 has 3482-byte rows).  `achieved` divides
+    # the step's FLOPs by the step's time, so it includes the repack.
     peak = peaks.get("bf16_tflops") or fallback_peaks()["bf16_tflops"]
     achieved = fl_step / (t / args.steps) / 1e12
-    traffic = recorded_traffic("umma_gemm_prefill_q_proj.txt")
+    traffic = recorded_traffic("chain_prefill_q_proj.txt")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_kind": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
-                "kernel": "umma_gemm_kernel x2 per step (GEMM1 T=X·A, GEMM2 Y=T·B)",
+                "kernel": "umma_chain_kernel (GEMM1 + GEMM2, one launch) + repack_chunks_kernel (A) per step; achieved = step FLOPs / step time",
                 "algorithmic_bytes_per_step": acc.algorithmic_bytes(M, K, R, N),
                 "flops_per_step": fl_step}
 

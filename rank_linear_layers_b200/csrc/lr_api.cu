@@ -49,8 +49,36 @@ struct Workspace {
   // Split-K partial sums of the chain kernel (fp32, zero at rest).
   float* split_ws = nullptr;
   size_t split_cap = 0;
+  // The prefill path's realigned operands, in two areas used by alternate
+  // calls (a call's repack may overlap the previous call's chain launch).
+  char* rp_area[2] = {nullptr, nullptr};
+  size_t rp_cap = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+// What the library last launched on a stream: whether it was a prefill
+// chain launch (whose output Y is known), and the parity that alternates the
+// prefill path's two realignment areas between calls.
+struct StreamState {
+  bool last_chain = false;
+  uintptr_t y_lo[4] = {0, 0, 0, 0}, y_hi[4] = {0, 0, 0, 0};  // last outputs written
+  unsigned int n_out = 0;
+  unsigned int parity = 0;
+  long long launches_after = -1;  // library launch count right after that launch
+};
+std::map<std::pair<int, cudaStream_t>, StreamState> g_streams;
+
+void note_call(cudaStream_t stream, bool chain, const void* y, size_t ybytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  StreamState& st = g_streams[{dev, stream}];
+  st.last_chain = chain;
+  st.launches_after = chain ? g_launches.load() : -1;
+  const unsigned int i = (st.n_out++) & 3u;
+  st.y_lo[i] = reinterpret_cast<uintptr_t>(y);
+  st.y_hi[i] = st.y_lo[i] + ybytes;
+}
 
 struct Staging {
   char* ptr = nullptr;
@@ -335,6 +363,43 @@ lr_status chain_split_ws(cudaStream_t stream, size_t bytes, float** out) {
   return LR_OK;
 }
 
+// The realignment area of this prefill call on `stream` (`bytes` each, the
+// two areas alternating between calls), and whether the call's first repack
+// may read its sources while the previous launch on the stream still runs:
+// only if that launch is the library's own prefill chain launch and none of
+// the last four outputs the library wrote on the stream overlaps `srcs`.
+lr_status repack_area(cudaStream_t stream, size_t bytes,
+                      std::initializer_list<std::pair<const void*, size_t>> srcs, char** area,
+                      bool* early) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  StreamState& ss = g_streams[{dev, stream}];
+  if (bytes > w.rp_cap) {
+    LR_CUDA(cudaStreamSynchronize(stream));
+    for (char*& a : w.rp_area) {
+      if (a) LR_CUDA(cudaFree(a));
+      a = nullptr;
+    }
+    w.rp_cap = 0;
+    const size_t cap = align_up(bytes + bytes / 4, 1 << 20);
+    for (char*& a : w.rp_area) LR_CUDA(cudaMalloc(&a, cap));
+    w.rp_cap = cap;
+  }
+  *area = w.rp_area[ss.parity & 1u];
+  ss.parity ^= 1u;
+  // ... and nothing else the library counts was launched since (any stream).
+  bool ok = ss.last_chain && ss.launches_after == g_launches.load();
+  for (const auto& sr : srcs) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(sr.first), hi = lo + sr.second;
+    for (int i = 0; i < 4; ++i)
+      if (sr.second && lo < ss.y_hi[i] && ss.y_lo[i] < hi) ok = false;
+  }
+  *early = ok;
+  return LR_OK;
+}
+
 // One launch of the chain kernel under construction.
 struct ChainBuild {
   ChainMaps maps{};
@@ -590,8 +655,12 @@ size_t repack_bytes(const void* p, int64_t ld, int64_t rows, int64_t cols) {
 
 // `*repacks` counts the repack launches of the call so far: all but the first
 // may start early (programmatic dependent launch).
+// With `early`, the call's first repack may overlap the previous launch and
+// read its source before that launch ends (the caller has checked that the
+// previous launch does not write it).
 lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t ld, int64_t rows,
-                      int64_t cols, char** scratch, Operand* out, int* repacks) {
+                      int64_t cols, char** scratch, Operand* out, int* repacks,
+                      bool early = false) {
   if (tma_ok(p, ld)) {
     *out = Operand{p, ld};
     return LR_OK;
@@ -601,7 +670,8 @@ lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t
   *scratch += repack_bytes(p, ld, rows, cols);
   lr_status st = launched(launch_repack(static_cast<const __nv_bfloat16*>(p), ld,
                                         span_bytes(rows, cols, ld), dst, ldd, rows, cols, d->sms,
-                                        stream, *repacks > 0));
+                                        stream, *repacks > 0 || early, wait_ctl(d),
+                                        *repacks > 0 || early));
   if (st != LR_OK) return st;
   ++*repacks;
   *out = Operand{dst, ldd};
@@ -613,20 +683,30 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
                       int64_t N, int64_t ldy) {
   const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), 8));
   const size_t tbytes = align_up(static_cast<size_t>(M) * ldt * 2, 256);
-  const size_t need = tbytes + repack_bytes(X, K, M, K) + repack_bytes(A, r, K, r) +
-                      repack_bytes(B, N, r, N);
+  const size_t rp = repack_bytes(X, K, M, K) + repack_bytes(A, r, K, r) + repack_bytes(B, N, r, N);
+  const bool pairs = g_path.load() == 4;
   char *zero = nullptr, *scratch = nullptr;
-  lr_status st = workspace(stream, 0, need, &zero, &scratch);
+  lr_status st = workspace(stream, 0, tbytes + (pairs ? rp : 0), &zero, &scratch);
   if (st != LR_OK) return st;
   void* T = scratch;
   scratch += tbytes;
+  // Misaligned operands are realigned into an area of their own; the
+  // call's first repack may overlap the previous launch (see repack_area).
+  bool early = false;
+  if (rp > 0 && !pairs) {
+    st = repack_area(stream, rp,
+                     {{X, span_bytes(M, K, K)}, {A, span_bytes(K, r, r)}, {B, span_bytes(r, N, N)}},
+                     &scratch, &early);
+    if (st != LR_OK) return st;
+  }
   Operand x, a, b;
   int repacks = 0;
-  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x, &repacks)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a, &repacks)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b, &repacks)) != LR_OK) return st;
-  if (g_path.load() == 4) {
+  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x, &repacks, early)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a, &repacks, early)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b, &repacks, early)) != LR_OK) return st;
+  if (pairs) {
     // CTA-pair tiles: the two GEMMs as two launches.
+    note_call(stream, false, Y, span_bytes(M, N, ldy));
     st = gemm_pair(d, stream, x.p, x.ld, a.p, a.ld, T, ldt, nullptr, M, r, K);
     if (st != LR_OK) return st;
     return gemm_pair(d, stream, T, ldt, b.p, b.ld, Y, ldy, bias, M, N, r);
@@ -634,8 +714,9 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   // One launch: GEMM1 T = X·A signals counter group 0 per 128-row block;
   // GEMM2 Y = T·B + bias waits on it row block by row block.  The launch
   // may overlap the kernel before it: after this call's repacks only the
-  // repacked operands depend on that kernel; with no repack, it is the
-  // caller's previous kernel, which may have written any input.
+  // repacked operands depend on that kernel (the repacks finish after the
+  // launch before them); with no repack, it is the caller's previous kernel,
+  // which may have written any input.
   const bool after_repack = repacks > 0;
   auto dep = [&](const void* used, const void* given) { return !after_repack || used != given; };
   ChainBuild cb;
@@ -648,7 +729,9 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   if (st != LR_OK) return st;
   st = chain_problem(cb, mt, 0, mb, M, N, r, Y, ldy, bias, 0, -1, false, dep(b.p, B));
   if (st != LR_OK) return st;
-  return run_chain(d, stream, cb);
+  st = run_chain(d, stream, cb);
+  note_call(stream, st == LR_OK, Y, span_bytes(M, N, ldy));
+  return st;
 }
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
@@ -662,11 +745,16 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
   int dev = 0;
   st = device_info(&d, &dev);
   if (st != LR_OK) return st;
-  if (K == 0 || r == 0) return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), ldy, M, N,
-                                                         static_cast<const __nv_bfloat16*>(bias),
-                                                         stream));
+  if (K == 0 || r == 0) {
+    note_call(stream, false, Y, span_bytes(M, N, ldy));
+    return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), ldy, M, N,
+                                     static_cast<const __nv_bfloat16*>(bias), stream));
+  }
   const bool decode = (path == 1) || (path == 0 && M <= 16);
-  if (decode) return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+  if (decode) {
+    note_call(stream, false, Y, span_bytes(M, N, ldy));
+    return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+  }
   return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
 }
 
@@ -683,6 +771,7 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
 // launch) when the group does not fit one launch's tables.
 lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* projs, int n,
                             int64_t M) {
+  for (int i = 0; i < n; ++i) note_call(stream, false, projs[i].Y, span_bytes(M, projs[i].N, projs[i].ld_y));
   struct Set {
     const void* X;
     int64_t K;
@@ -757,7 +846,8 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
         const lr_proj& p = projs[i];
         stt = launched(launch_repack(static_cast<const __nv_bfloat16*>(p.A), p.r,
                                      span_bytes(p.K, p.r, p.r), cat + off[static_cast<size_t>(i)],
-                                     st.width, p.K, p.r, d->sms, stream, repacks > 0));
+                                     st.width, p.K, p.r, d->sms, stream, repacks > 0,
+                                     wait_ctl(d)));
         if (stt != LR_OK) return stt;
         ++repacks;
       }
@@ -835,6 +925,10 @@ bool y_disjoint(const lr_proj& p, const lr_proj& q, int64_t M) {
 void note_cuda_error(int e) { g_last_cuda_error = e; }
 
 void note_launches(int n) { g_launches += n; }
+
+void note_output(cudaStream_t stream, const void* y, size_t bytes) {
+  note_call(stream, false, y, bytes);
+}
 
 cudaError_t ensure_max_smem(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -954,6 +1048,7 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
   if (st != LR_OK) return st;
   if (M == 0 || N == 0) return LR_OK;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  note_call(stream, false, Y, span_bytes(M, N, N));
   DeviceInfo* d = nullptr;
   int dev = 0;
   st = device_info(&d, &dev);
@@ -1075,14 +1170,17 @@ lr_status lr_release_workspaces(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_ws) {
-    if (!kv.second.ptr && !kv.second.ctrs && !kv.second.split_ws) continue;
+    if (!kv.second.ptr && !kv.second.ctrs && !kv.second.split_ws && !kv.second.rp_area[0]) continue;
     cudaSetDevice(kv.first.first);
     cudaStreamSynchronize(kv.first.second);
     if (kv.second.ptr) cudaFree(kv.second.ptr);
     if (kv.second.ctrs) cudaFree(kv.second.ctrs);
     if (kv.second.split_ws) cudaFree(kv.second.split_ws);
+    for (char* a : kv.second.rp_area)
+      if (a) cudaFree(a);
   }
   g_ws.clear();
+  g_streams.clear();
   for (auto& kv : g_stage) {
     if (!kv.second.ptr) continue;
     cudaSetDevice(kv.first.first);

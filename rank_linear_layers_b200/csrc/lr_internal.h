@@ -14,6 +14,9 @@ namespace lr {
 // for lr_kernel_launch_count(), from entry points outside lr_api.cu.
 void note_cuda_error(int e);
 void note_launches(int n);
+// Record that an entry point outside lr_api.cu wrote [y, y + bytes) on
+// `stream` (the prefill path checks its inputs against recent outputs).
+void note_output(cudaStream_t stream, const void* y, size_t bytes);
 
 // Read and clear the status word of lr_linear_decode_static on the current
 // device (0 if that entry point was never used there).  Allocates nothing.
@@ -183,10 +186,15 @@ cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& args, int grid,
 // columns from cols up to the next multiple of 8 are written as zero).
 // src_bytes is the byte extent of the source from its first element.  With
 // `dependent`, the launch may start while the previous launch on the stream
-// (which must not touch dst) still runs, and completes after it.
+// (which must not touch dst) still runs, and completes after it.  Contiguous
+// sources go through shared memory with bulk copies (bounded waits: `wait`).
+// With `read_early` (contiguous sources only) the copy may read the source
+// before the previous launch has finished: only for a source that launch
+// does not write.  Either way the launch completes after the previous one.
 cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_bytes,
                           __nv_bfloat16* dst, int64_t ldd, int64_t rows, int64_t cols,
-                          int num_sms, cudaStream_t stream, bool dependent = false);
+                          int num_sms, cudaStream_t stream, bool dependent, WaitCtl wait,
+                          bool read_early = false);
 
 // Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0).
 cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
