@@ -137,6 +137,7 @@ struct ChainProblem {
   int tile_begin;    // index of the problem's first tile in the launch
   int map_a, map_b;  // indices into ChainMaps
   int a_col0;        // column of operand a where this problem's K range starts
+  int b_col0;        // column of operand b where this problem's N range starts
   __nv_bfloat16* c;
   int64_t ldc;
   const __nv_bfloat16* bias;

@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         };
         auto load_b = [&](int st, int kb) {
           for (int c = 0; c < nbox; ++c)
-            tma_load_2d(stage_b(st) + c * B_ATOM, mb, &full[st], n_blk * P.bn + c * 64,
+            tma_load_2d(stage_b(st) + c * B_ATOM, mb, &full[st], P.b_col0 + n_blk * P.bn + c * 64,
                         (kbase + kb) * BK);
         };
         const bool gated_a = P.dep_a || P.wait_group >= 0;

@@ -54,11 +54,22 @@ def test_decoder_layer_group(M, n_int):
         # prefill path; on the decode path fp32 atomics may add partial sums
         # in another order, so compare at the parity tolerance there.
         A, B = dev[n]
-        Y1 = to_f64(lr.lr_linear(xs[p["x"]], A, B))
-        torch.cuda.synchronize()
         if M > 16:
+            # Without split K the single call does the same arithmetic per
+            # output element (tiling differs, sums do not); with split K
+            # (the default) fp32 reductions may add partial sums in another
+            # order.
+            lr.set_split_k(False)
+            try:
+                Y1 = to_f64(lr.lr_linear(xs[p["x"]], A, B))
+                torch.cuda.synchronize()
+            finally:
+                lr.set_split_k(True)
             assert np.array_equal(Y1, outs[n]), f"group vs single differ for {n}"
+            compare(to_f64(lr.lr_linear(xs[p["x"]], A, B))[rows], Yr, f"single {n} (split K)")
         else:
+            Y1 = to_f64(lr.lr_linear(xs[p["x"]], A, B))
+            torch.cuda.synchronize()
             compare(outs[n], Y1, f"group vs single {n}")
 
 
