@@ -146,21 +146,30 @@ __global__ void __launch_bounds__(kFmaWarps * 32, 2) skinny_fma_kernel(SkinnyArg
     return all_fast ? ld_nc_v4(c) : chunk16(c, a.w_lo, a.w_hi);
   };
 
+  // V's slice into shared memory (duplicated pairs) and zeroed partial sums.
+  auto stage_v = [&]() {
+    for (int m = 0; m < MT; ++m)
+      for (int kk = threadIdx.x; kk < a.k_chunk; kk += blockDim.x) {
+        const float v = (m < a.M && kk < kc) ? load_v(a, m, k0 + kk) : 0.f;
+        sv2[kk * MT + m] = make_float2(v, v);
+      }
+    for (int i = threadIdx.x; i < MT * CB; i += blockDim.x) part[i] = 0.f;
+    __syncthreads();
+  };
+
   // Rolling pipeline: U rows in flight; consuming row j issues row j + U
-  // into the same register slot.  The first U rows of W do not depend on V,
-  // so they are in flight before waiting for the launch that writes V.
+  // into the same register slot.  When V is written by the previous launch,
+  // the first U rows of W (which do not depend on V) are in flight before
+  // waiting for it; otherwise V is staged first, so that its few loads do not
+  // queue behind the CTA's (and the whole grid's) loads of W.
   uint4 cur[U];
+  if (!a.after_previous) stage_v();
 #pragma unroll
   for (int u = 0; u < U; ++u) cur[u] = load_row(u);
-  if (a.after_previous) griddep_wait();
-
-  for (int m = 0; m < MT; ++m)
-    for (int kk = threadIdx.x; kk < a.k_chunk; kk += blockDim.x) {
-      const float v = (m < a.M && kk < kc) ? load_v(a, m, k0 + kk) : 0.f;
-      sv2[kk * MT + m] = make_float2(v, v);
-    }
-  for (int i = threadIdx.x; i < MT * CB; i += blockDim.x) part[i] = 0.f;
-  __syncthreads();
+  if (a.after_previous) {
+    griddep_wait();
+    stage_v();
+  }
 
   float2 acc[MT][4];
 #pragma unroll
@@ -316,14 +325,10 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[t][i] = 0.f;
 
-  // The first k-steps' rows of W do not depend on V: issue them before
-  // waiting for the launch that writes V.
-  uint4 c_a[4], c_b[4], c_c[4];
-  mma_issue(w, 0, c_a);
-  mma_issue(w, 1, c_b);
-  mma_issue(w, 2, c_c);
-  if (a.after_previous) griddep_wait();
-
+  // When V is written by the previous launch, the first k-steps' rows of W
+  // (which do not depend on V) are issued before waiting for it; otherwise V
+  // is staged first, so that its loads do not queue behind W's.
+  auto stage_v = [&]() {
   // Fragment element e of lane f (g = f/4, tq = f%4) for residue res and
   // k-step j: token g or g+8, local row res + 8·(16j + i) with
   // i in {2tq, 2tq+1, 2tq+8, 2tq+9} (the mma.m16n8k16 A layout).
@@ -356,6 +361,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
   }
   for (int i = threadIdx.x; i < 16 * CB; i += blockDim.x) part[i] = 0.f;
   __syncthreads();
+  };
+  uint4 c_a[4], c_b[4], c_c[4];
+  if (!a.after_previous) stage_v();
+  mma_issue(w, 0, c_a);
+  mma_issue(w, 1, c_b);
+  mma_issue(w, 2, c_c);
+  if (a.after_previous) {
+    griddep_wait();
+    stage_v();
+  }
 
   for (int j = 0; j < nsteps; j += kMmaInflight) {
     mma_consume<V_F32>(w, j, c_a, tbuf, sfrag, res, d);

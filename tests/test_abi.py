@@ -90,6 +90,16 @@ def test_controls(L):
     assert L.lr_set_wait_limit_ns(-1) == lr.LR_ERR_INVALID_ARG
     assert L.lr_set_wait_limit_ns(0) == lr.LR_OK
     assert L.lr_kernel_launch_count() >= 0
+    # Tile width: 0 (automatic) or a multiple of 32 up to 256.
+    for bad in (-32, 16, 48, 257, 288):
+        assert L.lr_set_tile_n(bad) == lr.LR_ERR_INVALID_ARG
+    for ok in (32, 96, 256, 0):
+        assert L.lr_set_tile_n(ok) == lr.LR_OK
+    for bad in (-1, 2):
+        assert L.lr_set_split_k(bad) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_set_split_k(0) == lr.LR_OK and L.lr_set_split_k(1) == lr.LR_OK
+    assert L.lr_set_withhold_first_stage(2) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_set_withhold_first_stage(0) == lr.LR_OK
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
