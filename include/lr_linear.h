@@ -64,8 +64,18 @@ typedef enum {
  * K == 0 or r == 0: the sum is empty and Y = bias (or 0).
  *
  * Path: M <= 16 takes the decode kernels (bandwidth-bound streaming of A then
- * B, T kept in fp32); larger M takes the tcgen05 prefill kernels (T = X·A
- * written once as bf16, then Y = T·B).  Neither path pads r on the host.
+ * B, T kept in fp32); larger M takes the tcgen05 prefill path: one launch
+ * computes T = X·A (written once as bf16) and Y = T·B, GEMM2's tiles
+ * waiting for GEMM1's rows inside the launch.  Neither path pads r on the
+ * host.  Prefill operands whose rows do not start on 32-byte boundaries
+ * (for instance A with r not a multiple of 16) are first copied to a
+ * 128-byte row pitch by the library; that copy may start while the previous
+ * launch on `stream` still runs only when that launch was this library's
+ * prefill launch, nothing else of the library was launched since, and
+ * none of the library's last four outputs on the stream overlaps the
+ * copied operand.  Results are deterministic except that split K (small
+ * prefill GEMMs, see lr_set_split_k) adds fp32 partial sums in a
+ * run-dependent order.
  */
 lr_status lr_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
                     int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
@@ -91,10 +101,16 @@ typedef struct {
 /*
  * lr_linear_group — every projection of `projs` (n_proj >= 0) on the same M,
  * in one call, on `stream`.  Each projection's result equals lr_linear on its
- * own arguments.  The Y ranges (rows × [0, N) at stride ld_y) of different
- * projections must not overlap each other or any input.  FlashSVD v1.5's
- * abstract describes the packed execution of a layer's projections this
- * mirrors (catalogue record of arXiv 2605.08314).
+ * own arguments (bit for bit when split K is off; otherwise up to the order
+ * of fp32 partial sums).  The Y ranges (rows × [0, N) at stride ld_y) of
+ * different projections must not overlap each other or any input.
+ * At M > 16 the group is one prefill launch when it fits the launch's tables
+ * (at most 12 GEMMs: one per set of projections sharing X, plus one per
+ * projection): projections with the same X pointer and K are one GEMM1 over
+ * their A factors copied side by side; otherwise, and at M <= 16, the
+ * projections run one by one.  FlashSVD v1.5's abstract describes the packed
+ * execution of a layer's projections this mirrors (catalogue record of
+ * arXiv 2605.08314).
  */
 lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream);
 
