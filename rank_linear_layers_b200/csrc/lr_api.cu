@@ -65,16 +65,19 @@ struct StreamState {
   unsigned int n_out = 0;
   unsigned int parity = 0;
   long long launches_after = -1;  // library launch count right after that launch
+  bool full_grid = false;         // that launch had a CTA on every SM
 };
 std::map<std::pair<int, cudaStream_t>, StreamState> g_streams;
 
-void note_call(cudaStream_t stream, bool chain, const void* y, size_t ybytes) {
+void note_call(cudaStream_t stream, bool chain, const void* y, size_t ybytes,
+               bool full_grid = false) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return;
   std::lock_guard<std::mutex> lk(g_mu);
   StreamState& st = g_streams[{dev, stream}];
   st.last_chain = chain;
   st.launches_after = chain ? g_launches.load() : -1;
+  st.full_grid = chain && full_grid;
   const unsigned int i = (st.n_out++) & 3u;
   st.y_lo[i] = reinterpret_cast<uintptr_t>(y);
   st.y_hi[i] = st.y_lo[i] + ybytes;
@@ -379,8 +382,11 @@ lr_status chain_split_ws(cudaStream_t stream, size_t bytes, float** out) {
 // The realignment area of this prefill call on `stream` (`bytes` each, the
 // two areas alternating between calls), and whether the call's first repack
 // may read its sources while the previous launch on the stream still runs:
-// only if that launch is the library's own prefill chain launch and none of
-// the last four outputs the library wrote on the stream overlaps `srcs`.
+// only if that launch is the library's own prefill chain launch with a CTA
+// on every SM (so that when all of its CTAs have started — which is when the
+// copy may start — every CTA of the launch before it, which may still read
+// the other area, has left), and none of the last four outputs the library
+// wrote on the stream overlaps `srcs`.
 lr_status repack_area(cudaStream_t stream, size_t bytes,
                       std::initializer_list<std::pair<const void*, size_t>> srcs, char** area,
                       bool* early) {
@@ -403,7 +409,7 @@ lr_status repack_area(cudaStream_t stream, size_t bytes,
   *area = w.rp_area[ss.parity & 1u];
   ss.parity ^= 1u;
   // ... and nothing else the library counts was launched since (any stream).
-  bool ok = ss.last_chain && ss.launches_after == g_launches.load();
+  bool ok = ss.last_chain && ss.full_grid && ss.launches_after == g_launches.load();
   for (const auto& sr : srcs) {
     const uintptr_t lo = reinterpret_cast<uintptr_t>(sr.first), hi = lo + sr.second;
     for (int i = 0; i < 4; ++i)
@@ -759,7 +765,7 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   st = chain_problem(cb, mt, 0, mb, M, N, r, Y, ldy, bias, 0, -1, false, dep(b.p, B));
   if (st != LR_OK) return st;
   st = run_chain(d, stream, cb);
-  note_call(stream, st == LR_OK, Y, span_bytes(M, N, ldy));
+  note_call(stream, st == LR_OK, Y, span_bytes(M, N, ldy), cb.args.total_tiles >= d->sms);
   return st;
 }
 
