@@ -455,7 +455,7 @@ def run_ours(args):
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_kind": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
-                "kernel": "umma_chain_kernel (GEMM1 + GEMM2, one launch) + repack_chunks_kernel (A) per step; achieved = step FLOPs / step time",
+                "kernel": "umma_chain_kernel (GEMM1 + GEMM2, one launch) + repack_rows_bulk_kernel (A) per step; achieved = step FLOPs / step time",
                 "algorithmic_bytes_per_step": acc.algorithmic_bytes(M, K, R, N),
                 "flops_per_step": fl_step}
 
@@ -560,6 +560,8 @@ def main():
                     help="only the misalignment sweep r = 1000..1100 and {64,128,512,2048}")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed prefill steps (for ncu captures); numbers are not a bench line")
+    ap.add_argument("--profile-decode", type=int, default=0, metavar="M",
+                    help="only decode steps of the gate/up shape at this M (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -567,7 +569,36 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep()
+    if args.profile_decode:
+        return run_profile_decode(args)
     return run_ours(args)
+
+
+def run_profile_decode(args):
+    """Decode steps of the gate/up shape (K 4096, r 2867, N 14336) at M =
+    args.profile_decode, for ncu captures of this command: warmup + steps
+    calls on one set of inputs, no timing line."""
+    import torch
+    import rank_linear_layers_b200 as lr
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    _, dk, dr, dn = DECODE_SHAPES[0]
+    dm = args.profile_decode
+    q = lrgen.lowrank_problem(dm, dk, dr, dn, seed=0)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    Xd, Ad, Bd = to_dev(q["X"]), to_dev(q["A"]), to_dev(q["B"])
+    Yd = torch.empty((dm, dn), dtype=torch.bfloat16, device=dev)
+    launches0 = lr.kernel_launch_count()
+    for _ in range(args.warmup + args.steps):
+        lr.lr_linear(Xd, Ad, Bd, None, Y=Yd)
+    torch.cuda.synchronize()
+    status = lr.last_device_status()
+    print(json.dumps({"profile_run": "decode", "M": dm, "K": dk, "r": dr, "N": dn,
+                      "gpu_launches": int(lr.kernel_launch_count() - launches0),
+                      "status": int(status)}))
+    return 0 if status == lr.LR_OK else 1
 
 
 def run_sweep():

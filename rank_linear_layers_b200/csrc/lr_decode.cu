@@ -52,6 +52,14 @@ constexpr int kMmaStepRows = 16 * kRes;  // rows covered by one k-step of all re
 constexpr int kMmaRowBytes = 8 * 16 + 16;  // 8 chunks per warp row, padded for ldmatrix
 constexpr int kMmaBufBytes = 16 * kMmaRowBytes;
 constexpr int kMmaInflight = 3;  // k-steps whose loads are in flight per warp
+// V is staged through the transpose buffers in blocks of kMmaRawK values of
+// k (rows padded to kMmaRawLd floats: at most 2-way bank conflicts when the
+// fragments are read back).
+constexpr int kMmaRawK = 512;
+constexpr int kMmaRawLd = kMmaRawK + 2;
+static_assert(kMmaRawK % kMmaStepRows == 0, "raw blocks hold whole k-steps");
+static_assert(16 * kMmaRawLd * 4 <= kMmaWarps * kMmaBufBytes, "raw block fits the buffers");
+static_assert((16 * kMmaRawK) % (kMmaWarps * 32) == 0, "whole loads per thread");
 
 
 constexpr int kSkinnyMaxSmem = 200 * 1024;
@@ -325,28 +333,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[t][i] = 0.f;
 
-  // When V is written by the previous launch, the first k-steps' rows of W
-  // (which do not depend on V) are issued before waiting for it; otherwise V
-  // is staged first, so that its loads do not queue behind W's.
-  auto stage_v = [&]() {
-  // Fragment element e of lane f (g = f/4, tq = f%4) for residue res and
+  // V's slice is staged as the warps read it: sfrag[j][res][lane] holds
+  // fragment element e of lane f (g = f/4, tq = f%4) for residue res and
   // k-step j: token g or g+8, local row res + 8·(16j + i) with
-  // i in {2tq, 2tq+1, 2tq+8, 2tq+9} (the mma.m16n8k16 A layout).
-  const int nfrag = (a.k_chunk / kMmaStepRows) * kRes * 32;
-  for (int idx = threadIdx.x; idx < nfrag; idx += blockDim.x) {
-    const int f = idx & 31, rs = (idx >> 5) & (kRes - 1), j = idx >> 8;
-    const int g = f >> 2, tq = f & 3;
-    const int ii[4] = {2 * tq, 2 * tq + 1, 2 * tq + 8, 2 * tq + 9};
-    float v[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int kk = rs + kRes * (16 * j + ii[q]);
-      const bool in = kk < kc;
-      // order: (g, i0) (g, i1) (g+8, i0) (g+8, i1) (g, i8) (g, i9) (g+8, i8) (g+8, i9)
-      const int slot = (q < 2) ? q : 4 + (q - 2);
-      v[slot] = (in && g < a.M) ? load_v(a, g, k0 + kk) : 0.f;
-      v[slot + 2] = (in && g + 8 < a.M) ? load_v(a, g + 8, k0 + kk) : 0.f;
-    }
+  // i in {2tq, 2tq+1, 2tq+8, 2tq+9} (the mma.m16n8k16 A layout), as a bf16
+  // hi part and a bf16 lo part (the rounding error of hi; zero for bf16 V).
+  auto put_frag = [&](int gi, const float (&v)[8]) {
     uint4 hi, lo;
     hi.x = pack_bf16x2(v[0], v[1]);
     hi.y = pack_bf16x2(v[2], v[3]);
@@ -356,12 +348,82 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1) skinny_mma_kernel(SkinnyArg
     lo.y = pack_bf16x2(v[2] - bf16lo_to_f32(hi.y), v[3] - bf16hi_to_f32(hi.y));
     lo.z = pack_bf16x2(v[4] - bf16lo_to_f32(hi.z), v[5] - bf16hi_to_f32(hi.z));
     lo.w = pack_bf16x2(v[6] - bf16lo_to_f32(hi.w), v[7] - bf16hi_to_f32(hi.w));
-    sfrag[2 * idx] = hi;
-    sfrag[2 * idx + 1] = lo;
-  }
-  for (int i = threadIdx.x; i < 16 * CB; i += blockDim.x) part[i] = 0.f;
-  __syncthreads();
+    sfrag[2 * gi] = hi;
+    sfrag[2 * gi + 1] = lo;
   };
+  // Order of one fragment's elements: (g, i0) (g, i1) (g+8, i0) (g+8, i1)
+  // (g, i8) (g, i9) (g+8, i8) (g+8, i9).
+  // Direct: each element loaded from V in fragment order (bf16 V: the
+  // scattered loads mostly hit L1).
+  auto stage_direct = [&]() {
+    const int nfrag = (a.k_chunk / kMmaStepRows) * kRes * 32;
+    for (int idx = threadIdx.x; idx < nfrag; idx += blockDim.x) {
+      const int f = idx & 31, rs = (idx >> 5) & (kRes - 1), j = idx >> 8;
+      const int g = f >> 2, tq = f & 3;
+      const int ii[4] = {2 * tq, 2 * tq + 1, 2 * tq + 8, 2 * tq + 9};
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = rs + kRes * (16 * j + ii[q]);
+        const bool in = kk < kc;
+        const int slot = (q < 2) ? q : 4 + (q - 2);
+        v[slot] = (in && g < a.M) ? load_v(a, g, k0 + kk) : 0.f;
+        v[slot + 2] = (in && g + 8 < a.M) ? load_v(a, g + 8, k0 + kk) : 0.f;
+      }
+      put_frag(idx, v);
+    }
+  };
+  // Blocked (fp32 V, read from L2 one 32-byte sector per element when loaded
+  // in fragment order): through the still idle transpose buffers in blocks
+  // of kMmaRawK values of k, coalesced loads into raw[16][kMmaRawLd] (zero
+  // outside M and kc), then the fragments of the block's k-steps from there.
+  auto stage_blocked = [&]() {
+    constexpr int kThreads = kMmaWarps * 32;
+    constexpr int kPer = 16 * kMmaRawK / kThreads;
+    float* raw = reinterpret_cast<float*>(bufs);
+    for (int kb = 0; kb < a.k_chunk; kb += kMmaRawK) {
+      float t[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = threadIdx.x + u * kThreads;
+        const int m = idx / kMmaRawK, kk = kb + idx % kMmaRawK;
+        t[u] = (m < a.M && kk < kc) ? load_v(a, m, k0 + kk) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = threadIdx.x + u * kThreads;
+        raw[(idx / kMmaRawK) * kMmaRawLd + idx % kMmaRawK] = t[u];
+      }
+      __syncthreads();
+      const int j0 = kb / kMmaStepRows;
+      const int span = (a.k_chunk - kb < kMmaRawK) ? a.k_chunk - kb : kMmaRawK;
+      const int nfrag = (span / kMmaStepRows) * kRes * 32;
+      for (int idx = threadIdx.x; idx < nfrag; idx += kThreads) {
+        const int f = idx & 31, rs = (idx >> 5) & (kRes - 1), jl = idx >> 8;
+        const int g = f >> 2, tq = f & 3;
+        const int ii[4] = {2 * tq, 2 * tq + 1, 2 * tq + 8, 2 * tq + 9};
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int kl = rs + kRes * (16 * jl + ii[q]);
+          const int slot = (q < 2) ? q : 4 + (q - 2);
+          v[slot] = raw[g * kMmaRawLd + kl];
+          v[slot + 2] = raw[(g + 8) * kMmaRawLd + kl];
+        }
+        put_frag(j0 * kRes * 32 + idx, v);
+      }
+      __syncthreads();  // raw is refilled by the next block
+    }
+  };
+  auto stage_v = [&]() {
+    if (V_F32) stage_blocked();
+    else stage_direct();
+    for (int i = threadIdx.x; i < 16 * CB; i += blockDim.x) part[i] = 0.f;
+    __syncthreads();
+  };
+  // When V is written by the previous launch, the first k-steps' rows of W
+  // (which do not depend on V) are issued before waiting for it; otherwise V
+  // is staged first, so that its loads do not queue behind W's.
   uint4 c_a[4], c_b[4], c_c[4];
   if (!a.after_previous) stage_v();
   mma_issue(w, 0, c_a);
