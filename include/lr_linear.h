@@ -69,13 +69,18 @@ typedef enum {
  * waiting for GEMM1's rows inside the launch.  Neither path pads r on the
  * host.  Prefill operands whose rows do not start on 32-byte boundaries
  * (for instance A with r not a multiple of 16) are first copied to a
- * 128-byte row pitch by the library; that copy may start while the previous
- * launch on `stream` still runs only when that launch was this library's
- * prefill launch, nothing else of the library was launched since, and
- * none of the library's last four outputs on the stream overlaps the
- * copied operand.  Results are deterministic except that split K (small
- * prefill GEMMs, see lr_set_split_k) adds fp32 partial sums in a
- * run-dependent order.
+ * 128-byte row pitch by the library.  That copy, and the loads of the
+ * operands that need none, may begin before the previous kernel on `stream`
+ * has finished (programmatic dependent launch) when, by the library's own
+ * record, its last launch was a prefill launch with a CTA on every SM,
+ * nothing else of the library was launched since, and none of its last
+ * four outputs on the stream overlaps X, A or B.  The library sees only its
+ * own launches: a kernel of the caller's, enqueued on `stream` between two
+ * calls, is waited for in full unless it lets its dependents start early
+ * (griddepcontrol.launch_dependents); a caller whose such kernels write X,
+ * A or B of the next call turns the early copy off (lr_set_early_copy).
+ * Results are deterministic except that split K (small prefill GEMMs, see
+ * lr_set_split_k) adds fp32 partial sums in a run-dependent order.
  */
 lr_status lr_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
                     int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
@@ -192,12 +197,19 @@ int lr_last_cuda_error(void);
  *   splits its K loop over several CTAs, which add fp32 partial sums into a
  *   workspace; the last one rounds and stores.  on = 0 turns it off (for
  *   tests and tuning); other values return LR_ERR_INVALID_ARG.
- * All four are process-wide and take effect on the next call.
+ * lr_set_early_copy — on = 1 (the default): a prefill call's realignment
+ *   copy may overlap the library's previous prefill launch on the stream
+ *   (conditions under lr_linear).  on = 0: every call's first copy waits
+ *   for all earlier work on the stream, so a caller's kernel that starts
+ *   its dependents early can safely write the next call's operands.  Other
+ *   values return LR_ERR_INVALID_ARG.
+ * All five are process-wide and take effect on the next call.
  */
 lr_status lr_set_path(int path);
 lr_status lr_set_wait_limit_ns(int64_t ns);
 lr_status lr_set_tile_n(int bn);
 lr_status lr_set_split_k(int on);
+lr_status lr_set_early_copy(int on);
 
 /*
  * lr_set_withhold_first_stage — testing failure detection only.  With on = 1,

@@ -32,7 +32,7 @@ EXPORTS = (
     "lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense", "lr_last_device_status",
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
     "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
-    "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k",
+    "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy",
 )
 
 
@@ -79,6 +79,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_set_withhold_first_stage.argtypes = [ctypes.c_int]
     L.lr_set_tile_n.argtypes = [ctypes.c_int]
     L.lr_set_split_k.argtypes = [ctypes.c_int]
+    L.lr_set_early_copy.argtypes = [ctypes.c_int]
     L.lr_kernel_launch_count.argtypes = []
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
@@ -86,7 +87,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
                  "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces", "lr_set_withhold_first_stage",
-                 "lr_set_tile_n", "lr_set_split_k"):
+                 "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy"):
         getattr(L, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = L
@@ -221,6 +222,13 @@ def set_tile_n(bn: int):
 def set_split_k(on: bool):
     """Split long K loops of small prefill GEMMs over several CTAs (default on)."""
     _check(lib().lr_set_split_k(1 if on else 0), "lr_set_split_k")
+
+
+def set_early_copy(on: bool):
+    """Let a prefill call's realignment copy overlap the library's previous
+    prefill launch on the stream (default on); off when the caller's own
+    kernels between calls write operands and start their dependents early."""
+    _check(lib().lr_set_early_copy(1 if on else 0), "lr_set_early_copy")
 
 
 def set_withhold_first_stage(on: bool):

@@ -26,6 +26,7 @@ std::atomic<long long> g_launches{0};
 std::atomic<int> g_withhold{0};
 std::atomic<int> g_tile_n{0};
 std::atomic<int> g_split_k{1};
+std::atomic<int> g_early_copy{1};
 constexpr long long kDefaultWaitNs = 2000000000LL;
 
 struct DeviceInfo {
@@ -386,7 +387,8 @@ lr_status chain_split_ws(cudaStream_t stream, size_t bytes, float** out) {
 // on every SM (so that when all of its CTAs have started — which is when the
 // copy may start — every CTA of the launch before it, which may still read
 // the other area, has left), and none of the last four outputs the library
-// wrote on the stream overlaps `srcs`.
+// wrote on the stream overlaps `srcs`, and the early copy is on
+// (lr_set_early_copy).
 lr_status repack_area(cudaStream_t stream, size_t bytes,
                       std::initializer_list<std::pair<const void*, size_t>> srcs, char** area,
                       bool* early) {
@@ -409,7 +411,8 @@ lr_status repack_area(cudaStream_t stream, size_t bytes,
   *area = w.rp_area[ss.parity & 1u];
   ss.parity ^= 1u;
   // ... and nothing else the library counts was launched since (any stream).
-  bool ok = ss.last_chain && ss.full_grid && ss.launches_after == g_launches.load();
+  bool ok = g_early_copy.load() != 0 && ss.last_chain && ss.full_grid &&
+            ss.launches_after == g_launches.load();
   for (const auto& sr : srcs) {
     const uintptr_t lo = reinterpret_cast<uintptr_t>(sr.first), hi = lo + sr.second;
     for (int i = 0; i < 4; ++i)
@@ -1187,6 +1190,12 @@ int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
 lr_status lr_set_split_k(int on) {
   if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
   g_split_k.store(on);
+  return LR_OK;
+}
+
+lr_status lr_set_early_copy(int on) {
+  if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
+  g_early_copy.store(on);
   return LR_OK;
 }
 

@@ -98,6 +98,9 @@ def test_controls(L):
     for bad in (-1, 2):
         assert L.lr_set_split_k(bad) == lr.LR_ERR_INVALID_ARG
     assert L.lr_set_split_k(0) == lr.LR_OK and L.lr_set_split_k(1) == lr.LR_OK
+    for bad in (-1, 2):
+        assert L.lr_set_early_copy(bad) == lr.LR_ERR_INVALID_ARG
+    assert L.lr_set_early_copy(0) == lr.LR_OK and L.lr_set_early_copy(1) == lr.LR_OK
     assert L.lr_set_withhold_first_stage(2) == lr.LR_ERR_INVALID_ARG
     assert L.lr_set_withhold_first_stage(0) == lr.LR_OK
 
