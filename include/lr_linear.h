@@ -52,7 +52,8 @@ typedef enum {
   LR_ERR_UNSUPPORTED = 2,  /* no sm_100 device, or a size beyond int32 tiles  */
   LR_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                */
   LR_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out               */
-  LR_ERR_NO_MEMORY = 5     /* workspace allocation failed                      */
+  LR_ERR_NO_MEMORY = 5,    /* workspace allocation failed                      */
+  LR_ERR_INFEASIBLE = 6    /* lr_gac_select: no selection fits the budget      */
 } lr_status;
 
 /*
@@ -220,6 +221,40 @@ lr_status lr_set_early_copy(int on);
  * written).  Nothing faults or hangs.  on = 0 (the default) turns it off.
  */
 lr_status lr_set_withhold_first_stage(int on);
+
+/*
+ * lr_gac_select — re-select the dimensions of n_items compressed weights
+ * under a parameter budget, as GAC does ("Why Smaller Is Slower?
+ * Dimensional Misalignment in Compressed LLMs", §4.3 Step 3: Constrained
+ * Optimization, and its budget-quantization paragraph).  Host memory and
+ * host code only; no GPU is needed.
+ *
+ * Weight i has n_cand[i] candidates (1..255; the aligned dimensions its
+ * dimension sweep, §4.2, kept), candidate j storing cost[off_i + j]
+ * parameters (off_i = n_cand[0] + … + n_cand[i-1]; 0 <= cost < 2^53), an
+ * importance score[i] (finite) and base[i] = |W_i*| (0 <= base < 2^53), the
+ * parameters at its unconstrained dimension.  The call picks one candidate
+ * per weight to maximise  Σ_i score[i]·(cost_i,choice[i] − base[i])  subject
+ * to  Σ_i ⌈cost_i,choice[i] / unit⌉ <= ⌊budget / unit⌋  (unit >= 1: the
+ * quantum u of the budget, e.g. 8·(smallest cost of one dimension step)),
+ * by the recurrence D[i][b] = max_j D[i−1][b − ⌈w_ij/u⌉] + v_ij with
+ * D[0][b] = 0.  Rounding costs up and the budget down keeps the selection's
+ * true parameter count within `budget`.  Among equally good candidates of a
+ * weight at a given remaining budget the lowest index is taken, so the
+ * result is deterministic.
+ *
+ * choice[n_items] receives the chosen candidate indices; *objective (may be
+ * NULL) the maximised sum, accumulated over the weights in order.
+ * Errors: LR_ERR_INVALID_ARG for null pointers, n_items < 1, counts, costs
+ * or scores out of range, budget < 0 or unit < 1; LR_ERR_INFEASIBLE when
+ * even the cheapest candidates exceed the quantized budget; LR_ERR_UNSUPPORTED
+ * when the table (n_items × (⌊budget/unit⌋ + 1) bytes) would exceed 1 GiB;
+ * LR_ERR_NO_MEMORY if host allocation fails.  choice is written only on
+ * LR_OK.
+ */
+lr_status lr_gac_select(int n_items, const int* n_cand, const int64_t* cost, const double* score,
+                        const int64_t* base, int64_t budget, int64_t unit, int* choice,
+                        double* objective);
 
 /* Counts the kernels launched by this library in this process. */
 int64_t lr_kernel_launch_count(void);

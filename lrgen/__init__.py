@@ -239,3 +239,28 @@ def decoder_layer(M: int, seed: int = 7, n_int: int = 14336, bias: bool = False)
         }
         projs[name] = p
     return {"M": M, "inputs": inputs, "projs": projs, "ranks": ranks, "n_int": n_int}
+
+
+def gac_model(layers: int = 32, seed: int = 11, n_int: int = 14336) -> list:
+    """Inputs for GAC's rank re-selection over `layers` decoder layers of the
+    Llama-3-8B projection shapes: per weight an unconstrained (fractional)
+    rank r* uniform on [0.35·m, 0.85·m], m = min(K, N), and an importance
+    score uniform on [0.5, 1.5), drawn weight by weight from counter streams
+    of ``seed`` (these stand in for a compressor's allocation and its
+    importance scores, which need trained weights)."""
+    out = []
+    idx = 0
+    for layer in range(layers):
+        for name, K, N, _ in LAYER_PROJECTIONS:
+            if name in ("gate", "up"):
+                N = n_int
+            if name == "down":
+                K = n_int
+            m = min(K, N)
+            c = np.array([idx], dtype=np.uint64)
+            u = uniform(seed, 901, c)[0]
+            s = uniform(seed, 902, c)[0]
+            out.append({"name": f"layers.{layer}.{name}", "K": K, "N": N,
+                        "r_star": float((0.35 + 0.5 * u) * m), "score": float(0.5 + s)})
+            idx += 1
+    return out

@@ -24,6 +24,7 @@ LR_ERR_UNSUPPORTED = 2
 LR_ERR_CUDA = 3
 LR_ERR_TIMEOUT = 4
 LR_ERR_NO_MEMORY = 5
+LR_ERR_INFEASIBLE = 6
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_PREFILL_1SM, PATH_PREFILL_PAIR = 0, 1, 2, 3, 4
 
@@ -33,6 +34,7 @@ EXPORTS = (
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
     "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
     "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy",
+    "lr_gac_select",
 )
 
 
@@ -80,6 +82,9 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_set_tile_n.argtypes = [ctypes.c_int]
     L.lr_set_split_k.argtypes = [ctypes.c_int]
     L.lr_set_early_copy.argtypes = [ctypes.c_int]
+    ip, lp, dp = (ctypes.POINTER(ctypes.c_int), ctypes.POINTER(i64),
+                  ctypes.POINTER(ctypes.c_double))
+    L.lr_gac_select.argtypes = [ctypes.c_int, ip, lp, dp, lp, i64, i64, ip, dp]
     L.lr_kernel_launch_count.argtypes = []
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
@@ -87,7 +92,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
                  "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces", "lr_set_withhold_first_stage",
-                 "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy"):
+                 "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy", "lr_gac_select"):
         getattr(L, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = L
@@ -229,6 +234,25 @@ def set_early_copy(on: bool):
     prefill launch on the stream (default on); off when the caller's own
     kernels between calls write operands and start their dependents early."""
     _check(lib().lr_set_early_copy(1 if on else 0), "lr_set_early_copy")
+
+
+def gac_select(costs: Sequence[Sequence[int]], scores: Sequence[float],
+               bases: Sequence[int], budget: int, unit: int):
+    """lr_gac_select: one candidate index per weight (costs[i][j] parameters)
+    maximising Σ scores[i]·(cost − bases[i]) within the quantized budget.
+    Returns (choices, objective); raises LrError (LR_ERR_INFEASIBLE when
+    nothing fits)."""
+    n = len(costs)
+    flat = [int(w) for c in costs for w in c]
+    n_cand = (ctypes.c_int * max(n, 1))(*[len(c) for c in costs])
+    cost = (ctypes.c_int64 * max(len(flat), 1))(*flat)
+    score = (ctypes.c_double * max(n, 1))(*[float(s) for s in scores])
+    base = (ctypes.c_int64 * max(n, 1))(*[int(b) for b in bases])
+    choice = (ctypes.c_int * max(n, 1))()
+    obj = ctypes.c_double()
+    _check(lib().lr_gac_select(n, n_cand, cost, score, base, int(budget), int(unit), choice,
+                               ctypes.byref(obj)), "lr_gac_select")
+    return [int(c) for c in choice[:n]], obj.value
 
 
 def set_withhold_first_stage(on: bool):

@@ -1167,6 +1167,7 @@ const char* lr_status_string(lr_status s) {
     case LR_ERR_CUDA: return "LR_ERR_CUDA";
     case LR_ERR_TIMEOUT: return "LR_ERR_TIMEOUT";
     case LR_ERR_NO_MEMORY: return "LR_ERR_NO_MEMORY";
+    case LR_ERR_INFEASIBLE: return "LR_ERR_INFEASIBLE";
   }
   return "LR_ERR_UNKNOWN";
 }
