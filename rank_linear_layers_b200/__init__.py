@@ -224,9 +224,11 @@ def set_tile_n(bn: int):
     _check(lib().lr_set_tile_n(bn), "lr_set_tile_n")
 
 
-def set_split_k(on: bool):
-    """Split long K loops of small prefill GEMMs over several CTAs (default on)."""
-    _check(lib().lr_set_split_k(1 if on else 0), "lr_set_split_k")
+def set_split_k(on):
+    """Split long K loops of small prefill GEMMs over several CTAs: False/0
+    off, True/1 on (the default), 2 also where the schedule model predicts a
+    shorter launch (experimental)."""
+    _check(lib().lr_set_split_k(int(on)), "lr_set_split_k")
 
 
 def set_early_copy(on: bool):
