@@ -13,7 +13,8 @@ FLOPs per step per rank, summed over ranks, over the max-over-ranks device
 time).  Inputs rotate over enough copies to exceed twice the L2 size, so no
 step reads its operands from L2.  Also reported: the roofline fraction of the
 prefill kernels, the end-to-end rate through the host-buffer C ABI call, the
-decode (M = 1, 4, 16) bandwidth of the Llama-3-8B MLP shapes, the fp64 CPU
+decode (M = 1, 4, 16) bandwidth of the Llama-3-8B MLP shapes, the time per
+call of the small single layer (16×256 · 256×107), the fp64 CPU
 oracle timed on a bounded sample (the CPU baseline), SM clocks sampled during
 the timed region and the number of library kernels launched.
 
@@ -316,6 +317,29 @@ def sweep_times(lr, dev, l2, ranks, steps=20, warmup=3):
     return out
 
 
+def single_layer_bench(lr, dev, steps=200, warmup=20):
+    """The small single layer, X [16,256] · A [256,107] · B [107,256] (seed 0,
+    no bias): launch- and latency-bound, so its absolute time per call is
+    the figure of merit.  Back-to-back calls on one stream, CUDA events."""
+    try:
+        import torch
+        q = lrgen.lowrank_problem(16, 256, 107, 256, seed=0)
+        X, A, B = (_dev_bits(q[k], dev) for k in ("X", "A", "B"))
+        Y = torch.empty((16, 256), dtype=torch.bfloat16, device=dev)
+        n0 = lr.kernel_launch_count()
+        lr.lr_linear(X, A, B, None, Y=Y)
+        per_call = lr.kernel_launch_count() - n0
+
+        def st(i):
+            lr.lr_linear(X, A, B, None, Y=Y)
+        t = time_steps(st, steps, warmup) / steps
+        return {"us_per_call": t * 1e6, "gpu_launches_per_call": int(per_call),
+                "flops": acc.flops(16, 256, 107, 256),
+                "note": "M=16 K=256 r=107 N=256, decode path, back-to-back calls"}
+    except Exception as ex:  # pragma: no cover - reported, not hidden
+        return {"error": str(ex)[:200]}
+
+
 def misalignment_check(lr, dev, l2, ranks=range(1000, 1009)):
     """Misaligned ranks against the nearest multiple of 8 (both neighbours
     at r = 4 mod 8), in time per FLOP."""
@@ -527,6 +551,7 @@ def run_ours(args):
         del Wd
     misalign = misalignment_check(lr, dev, l2) if not args.no_extra else None
     layer = layer_bench(lr, dev, peaks) if not args.no_extra else None
+    single = single_layer_bench(lr, dev) if not args.no_extra else None
 
     cb = cpu_baseline(p) if (rank == 0 and world == 1) else None
     if rank == 0:
@@ -537,7 +562,7 @@ def run_ours(args):
             "data": "synthetic", "config": config_dict(), "roofline": roofline,
             "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches_timed),
             "clocks": clk, "parity": parity, "decode": decode, "dense": dense,
-            "misalignment": misalign, "layer": layer,
+            "misalignment": misalign, "layer": layer, "single_layer": single,
         }
         print(json.dumps(line))
     if world > 1:
