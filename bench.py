@@ -551,6 +551,12 @@ def run_ours(args):
         del Wd
     misalign = misalignment_check(lr, dev, l2) if not args.no_extra else None
     layer = layer_bench(lr, dev, peaks) if not args.no_extra else None
+    layer_pruned = None
+    if not args.no_extra:
+        try:  # the pruned MLP (N_int = 12203: odd strides, 2-byte-aligned packed output)
+            layer_pruned = layer_bench(lr, dev, peaks, n_int=12203)
+        except Exception as ex:  # pragma: no cover - reported, not hidden
+            layer_pruned = {"error": str(ex)[:200]}
     single = single_layer_bench(lr, dev) if not args.no_extra else None
 
     cb = cpu_baseline(p) if (rank == 0 and world == 1) else None
@@ -562,7 +568,8 @@ def run_ours(args):
             "data": "synthetic", "config": config_dict(), "roofline": roofline,
             "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches_timed),
             "clocks": clk, "parity": parity, "decode": decode, "dense": dense,
-            "misalignment": misalign, "layer": layer, "single_layer": single,
+            "misalignment": misalign, "layer": layer, "layer_pruned": layer_pruned,
+            "single_layer": single,
         }
         print(json.dumps(line))
     if world > 1:
