@@ -489,6 +489,15 @@ def run_ours(args):
             print(json.dumps({"profile_run": True, "ms_per_step": ms, "gpu_launches": int(launches_timed)}))
         return 0
 
+    # Two more trials of the same K steps on this rank (the reported value is
+    # the first): the spread of the per-step time across trials.
+    trials = [t / args.steps * 1e3]
+    try:
+        for _ in range(2):
+            trials.append(time_steps(step, args.steps, 0) / args.steps * 1e3)
+    except Exception:  # pragma: no cover - the main figure stands alone
+        pass
+
     # End to end through the host-buffer C ABI call (pinned host memory).
     e2e = None
     try:
@@ -568,6 +577,8 @@ def run_ours(args):
             "data": "synthetic", "config": config_dict(), "roofline": roofline,
             "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches_timed),
             "clocks": clk, "parity": parity, "decode": decode, "dense": dense,
+            "trials_ms_per_step": trials,
+            "trial_spread_pct": (max(trials) - min(trials)) / statistics.median(trials) * 100,
             "misalignment": misalign, "layer": layer, "layer_pruned": layer_pruned,
             "single_layer": single,
         }
