@@ -603,6 +603,9 @@ def main():
                     help="only the misalignment sweep r = 1000..1100 and {64,128,512,2048}")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed prefill steps (for ncu captures); numbers are not a bench line")
+    ap.add_argument("--gac-sweep", action="store_true",
+                    help="only time lr_linear at the ranks the GAC planner sweeps, per weight shape")
+    ap.add_argument("--gac-m", type=int, default=2048, help="tokens for --gac-sweep")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="M",
                     help="only decode steps of the gate/up shape at this M (for ncu captures)")
     args = ap.parse_args()
@@ -614,6 +617,8 @@ def main():
         return run_sweep()
     if args.profile_decode:
         return run_profile_decode(args)
+    if args.gac_sweep:
+        return run_gac_sweep(args)
     return run_ours(args)
 
 
@@ -641,6 +646,45 @@ def run_profile_decode(args):
     print(json.dumps({"profile_run": "decode", "M": dm, "K": dk, "r": dr, "N": dn,
                       "gpu_launches": int(lr.kernel_launch_count() - launches0),
                       "status": int(status)}))
+    return 0 if status == lr.LR_OK else 1
+
+
+def run_gac_sweep(args):
+    """The GAC planner's dimension sweep (§4.2 of the GAC paper) on this GPU:
+    for each weight shape of the 32-layer Llama-3-8B-shaped model, the time
+    per lr_linear call at every rank the planner may choose, M = args.gac_m
+    tokens.  One JSON line: {"times_us": {"KxN": {rank: us}}}, the input of
+    ``python -m rank_linear_layers_b200.gac --times``.  X rotates over copies
+    larger than twice L2; A and B of a rank are the leading columns / rows of
+    one seeded draw."""
+    import torch
+    import rank_linear_layers_b200 as lr
+    from rank_linear_layers_b200 import gac
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ws = [gac.Weight(**d) for d in lrgen.gac_model(32, seed=11)]
+    Mw = args.gac_m
+    out = {}
+    for (Kw, Nw), ranks in sorted(gac.sweep_plan(ws).items()):
+        rmax = max(ranks)
+        X0 = _dev_bits(lrgen.normal_bf16(0, 1, (Mw, Kw)), dev)
+        Xs = [X0] + [X0.clone() for _ in range(max(1, math.ceil(2 * l2 / (X0.numel() * 2))))]
+        Af = _dev_bits(lrgen.normal_bf16(0, 2, (Kw, rmax), 1.0 / math.sqrt(Kw)), dev)
+        Bf = _dev_bits(lrgen.normal_bf16(0, 3, (rmax, Nw), 1.0 / math.sqrt(rmax)), dev)
+        Y = torch.empty((Mw, Nw), dtype=torch.bfloat16, device=dev)
+        t = {}
+        for r in ranks:
+            A = Af[:, :r].contiguous()
+            B = Bf[:r].contiguous()
+
+            def st(i, A=A, B=B):
+                lr.lr_linear(Xs[i % len(Xs)], A, B, None, Y=Y)
+            t[r] = round(time_steps(st, 20, 3) / 20 * 1e6, 3)
+        out[f"{Kw}x{Nw}"] = t
+        del Xs, Af, Bf, Y
+    status = lr.last_device_status()
+    print(json.dumps({"gac_sweep": True, "M": Mw, "times_us": out, "status": int(status)}))
     return 0 if status == lr.LR_OK else 1
 
 

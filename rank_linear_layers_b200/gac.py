@@ -5,7 +5,7 @@ GAC: GPU-Aligned Compression.  Step 1, the compressor's unconstrained
 allocation r_i*, happens upstream.  Step 2, the dimension sweep (§4.2),
 proposes aligned ranks near r_i* (``sweep_ranks``) and keeps those whose
 measured time on this GPU shows no cliff (``drop_cliffs``; the times come
-from timing lr_linear at each rank, as ``bench.py --sweep`` does).  Step 3
+from timing lr_linear at each rank, as ``bench.py --gac-sweep`` does).  Step 3
 (§4.3) picks one candidate per weight under the same parameter budget
 (``plan``, which calls lr_gac_select in the C library).
 
@@ -14,6 +14,8 @@ weight (r·(K+N) ≥ K·N) is replaced by the dense weight itself, the dense
 fallback the LowRankArena review describes for DoBi-SVD.
 
     python -m rank_linear_layers_b200.gac     # plans a 32-layer model, times it
+    python bench.py --gac-sweep > sweep.json  # per-shape rank timings on the GPU
+    python -m rank_linear_layers_b200.gac --times sweep.json
 """
 from __future__ import annotations
 
@@ -111,6 +113,28 @@ def candidates(w: Weight, times: Optional[Mapping[int, float]] = None, align: in
     return out
 
 
+def sweep_plan(weights: Sequence[Weight], align: int = 8, coarse: int = 4) -> dict:
+    """The ranks to time for each weight shape: {(K, N): sorted ranks}, the
+    union of the weights' swept ranks (one timing serves every weight of a
+    shape)."""
+    plan = {}
+    for w in weights:
+        plan.setdefault((w.K, w.N), set()).update(
+            sweep_ranks(w.r_star, align, coarse, limit=min(w.K, w.N)))
+    return {k: sorted(v) for k, v in plan.items()}
+
+
+def times_by_weight(weights: Sequence[Weight], shape_times: Mapping) -> dict:
+    """Per-weight rank timings from per-shape ones.  `shape_times` maps
+    "KxN" (as ``bench.py --gac-sweep`` writes it) or (K, N) to {rank: time}."""
+    out = {}
+    for w in weights:
+        t = shape_times.get(f"{w.K}x{w.N}", shape_times.get((w.K, w.N)))
+        if t:
+            out[w.name] = {int(r): float(v) for r, v in t.items()}
+    return out
+
+
 def budget_for(weights: Sequence[Weight]) -> int:
     """The compressor's own budget: Σ r_i*·(K_i + N_i), rounded down (GAC
     re-selects under the same parameter budget)."""
@@ -147,13 +171,24 @@ def _main() -> int:
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--seed", type=int, default=11)
     ap.add_argument("--repeat", type=int, default=5)
+    ap.add_argument("--times", help="JSON written by `bench.py --gac-sweep` (per-shape rank timings)")
+    ap.add_argument("--tol", type=float, default=0.05)
     args = ap.parse_args()
     ws = [Weight(**d) for d in lrgen.gac_model(args.layers, args.seed)]
+    wt = None
+    if args.times:
+        with open(args.times) as f:
+            wt = times_by_weight(ws, json.load(f)["times_us"])
     times = []
     for _ in range(args.repeat):
         t0 = time.perf_counter()
-        p = plan(ws)
+        p = plan(ws, times=wt, tol=args.tol)
         times.append(time.perf_counter() - t0)
+    cliffs = 0
+    if wt:
+        for w in ws:
+            swept = sweep_ranks(w.r_star, limit=min(w.K, w.N))
+            cliffs += len(swept) - len(drop_cliffs(swept, wt.get(w.name, {}), args.tol))
     unaligned = sum(1 for w in ws if abs(w.r_star - round(w.r_star)) > 0 or round(w.r_star) % 8)
     print(json.dumps({
         "weights": len(ws), "budget": p.budget, "unit": p.unit,
@@ -161,6 +196,7 @@ def _main() -> int:
         "objective": p.objective, "aligned_fraction": p.aligned_fraction,
         "unaligned_before": unaligned / len(ws),
         "dense_fallbacks": sum(1 for r in p.ranks.values() if r is DENSE),
+        "measured_times": bool(wt), "cliffs_dropped": cliffs,
         "plan_ms_median": sorted(times)[len(times) // 2] * 1e3}))
     return 0
 

@@ -231,3 +231,18 @@ def test_plan_keeps_the_budget_and_aligns_every_rank(L):
     with pytest.raises(lr.LrError) as e:
         gac.plan(ws, budget=1000)
     assert e.value.code == lr.LR_ERR_INFEASIBLE
+
+
+def test_sweep_plan_and_times_by_weight():
+    ws = [gac.Weight("a", 4096, 4096, 1000.0), gac.Weight("b", 4096, 4096, 1010.0),
+          gac.Weight("c", 4096, 1024, 300.0)]
+    sp = gac.sweep_plan(ws)
+    assert set(sp) == {(4096, 4096), (4096, 1024)}
+    assert sp[(4096, 4096)] == sorted(set(gac.sweep_ranks(1000.0, limit=4096))
+                                      | set(gac.sweep_ranks(1010.0, limit=4096)))
+    assert sp[(4096, 1024)] == gac.sweep_ranks(300.0, limit=1024)
+    shape_times = {"4096x4096": {str(r): 1.0 + r * 1e-3 for r in sp[(4096, 4096)]}}
+    wt = gac.times_by_weight(ws, shape_times)
+    assert set(wt) == {"a", "b"}  # no timings for the 4096x1024 shape
+    assert wt["a"][1000] == pytest.approx(2.0)
+    assert gac.times_by_weight(ws, {(4096, 1024): {304: 3.0}}) == {"c": {304: 3.0}}
