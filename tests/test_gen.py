@@ -106,3 +106,13 @@ def test_prefill_svd_construction_eckart_young():
     # The bf16 factors are the fp64 products rounded once.
     assert np.array_equal(p["A"], lrgen.bf16_bits(A64))
     assert np.array_equal(p["B"], lrgen.bf16_bits(B64))
+    # Statistical sanity of the workload: for X ~ N(0,1) a row of X·A·B has
+    # expected squared norm Σ_{i<=r} σ_i² (U and V orthogonal), so
+    # RMS(Y) = sqrt(Σ_{i<=r} (1/i) / N) ≈ 0.0443.  64 rows: the estimate's
+    # standard deviation is about 1.4%.
+    import oracle
+    X = lrgen.normal_bf16(0, 77, (64, K), 1.0)
+    Y = oracle.lr_linear(X, p["A"], p["B"])
+    expect = math.sqrt(head / N)
+    assert abs(expect - 0.0443) < 1e-4
+    assert abs(float(np.sqrt(np.mean(Y ** 2))) / expect - 1) < 0.06
