@@ -246,3 +246,15 @@ def test_sweep_plan_and_times_by_weight():
     assert set(wt) == {"a", "b"}  # no timings for the 4096x1024 shape
     assert wt["a"][1000] == pytest.approx(2.0)
     assert gac.times_by_weight(ws, {(4096, 1024): {304: 3.0}}) == {"c": {304: 3.0}}
+
+
+def test_c_solver_largest_candidate_index(L):
+    """255 candidates (the most a weight may have): the last index is
+    reachable and the result still equals the oracle's."""
+    costs = [list(range(0, 255 * 3, 3)), [5, 9]]
+    scores, bases = [1.0, 2.0], [100, 7]
+    for budget in (10 ** 6, 400, 9):
+        want = ref.select(costs, scores, bases, budget, 1)
+        got = lr.gac_select(costs, scores, bases, budget, 1)
+        assert got[0] == want[0] and got[1] == want[1]
+    assert lr.gac_select(costs, scores, bases, 10 ** 6, 1)[0] == [254, 1]
