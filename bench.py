@@ -237,13 +237,23 @@ def aggregate(flops_per_rank, seconds_per_rank, world):
 
 
 # ---------------------------------------------------------------- CPU baseline
-def cpu_baseline(p, budget_s=12.0):
-    """The fp64 oracle on a bounded row sample of the same workload."""
+def cpu_baseline(p, check=None, budget_s=12.0):
+    """The fp64 oracle on a bounded row sample of the same workload.  Its
+    first chunk is `check` = (rows, the GPU's bf16 output of those rows as
+    fp64), whose parity with the oracle is returned beside the timing."""
     import oracle
     threads = oracle.default_threads()
     rows_per_chunk = 32
     done = 0
+    parity = None
     t0 = time.perf_counter()
+    if check is not None:
+        rows, Yg = check
+        Yr = oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rows, threads=threads)
+        done += len(rows)
+        rms = float(np.sqrt(np.mean(Yr ** 2)))
+        parity = {"rows": int(len(rows)), "max_err_over_rms": float(np.abs(Yg - Yr).max() / rms),
+                  "rel_fro": float(np.linalg.norm(Yg - Yr) / np.linalg.norm(Yr))}
     rng = np.random.default_rng(1)
     while time.perf_counter() - t0 < budget_s and done < 4 * M:
         rows = rng.choice(M, rows_per_chunk, replace=False)
@@ -251,8 +261,9 @@ def cpu_baseline(p, budget_s=12.0):
         done += rows_per_chunk
     dt = time.perf_counter() - t0
     fl = acc.flops(done, K, R, N)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} rows of X (of {M}) through the fp64 oracle, {dt:.1f} s"}
+    cb = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+          "sample": f"{done} rows of X (of {M}) through the fp64 oracle, {dt:.1f} s"}
+    return cb, parity
 
 
 def run_reference(args):
@@ -436,20 +447,16 @@ def run_ours(args):
         j = i % copies
         lr.lr_linear(Xs[j], As[j], Bs[j], None, Y=Y)
 
-    # Correctness gate on the timed configuration: sampled rows vs the oracle.
+    # Correctness gate on the timed configuration: the device status now, and
+    # 16 sampled output rows kept for the CPU-baseline leg, which checks them
+    # against the oracle (rank 0, one GPU).
     step(0)
     torch.cuda.synchronize()
     if lr.last_device_status() != lr.LR_OK:
         raise RuntimeError("device status not OK")
-    parity = None
-    if rank == 0:
-        import oracle
-        rows = np.random.default_rng(0).choice(M, 16, replace=False)
-        Yr = oracle.lr_linear(p["X"], p["A"], p["B"], None, rows=rows)
-        Yg = lrgen.bf16_to_f64(Y[torch.as_tensor(rows, device=dev)].cpu().view(torch.int16).numpy().view(np.uint16))
-        rms = float(np.sqrt(np.mean(Yr ** 2)))
-        parity = {"rows": 16, "max_err_over_rms": float(np.abs(Yg - Yr).max() / rms),
-                  "rel_fro": float(np.linalg.norm(Yg - Yr) / np.linalg.norm(Yr))}
+    check_rows = np.random.default_rng(0).choice(M, 16, replace=False)
+    check_Y = lrgen.bf16_to_f64(
+        Y[torch.as_tensor(check_rows, device=dev)].cpu().view(torch.int16).numpy().view(np.uint16))
 
     clocks = ClockSampler(local)
     barrier(world)
@@ -568,7 +575,8 @@ def run_ours(args):
             layer_pruned = {"error": str(ex)[:200]}
     single = single_layer_bench(lr, dev) if not args.no_extra else None
 
-    cb = cpu_baseline(p) if (rank == 0 and world == 1) else None
+    cb, parity = (cpu_baseline(p, check=(check_rows, check_Y)) if (rank == 0 and world == 1)
+                  else (None, None))
     if rank == 0:
         line = {
             "metric": metric_name(), "value": value, "unit": "TFLOP/s", "n_gpus": world,

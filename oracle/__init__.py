@@ -1,7 +1,8 @@
 """CPU fp64 oracle for Y = (X·A)·B (+bias) — TEST INFRASTRUCTURE ONLY.
 
-Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  The product path (the CUDA library and
+Only ``tests/``, ``__graft_entry__.smoke()`` and, in ``bench.py``, the
+CPU-baseline leg (which also checks 16 sampled GPU rows) and the reference
+arm (``--impl reference``) may import this package.  The product path (the CUDA library and
 its Python binding) never imports, links or calls it, and shares no code with
 it.
 
