@@ -109,3 +109,29 @@ def test_controls(L):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         lr.lib(str(tmp_path / "missing.so"))
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/lr_linear.h compiles as C99 (-pedantic) and a C program links
+    against the library and calls it (the host-only planner entry point, so
+    no GPU is needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "lr_linear.h"\n'
+        "int main(void) {\n"
+        "  int n_cand[2] = {2, 1}; int64_t cost[3] = {8, 16, 24};\n"
+        "  double score[2] = {1.0, 1.0}; int64_t base[2] = {8, 24};\n"
+        "  int choice[2] = {-1, -1}; double obj = 0.0; lr_proj p = {0}; (void)p;\n"
+        "  if (lr_gac_select(2, n_cand, cost, score, base, 40, 8, choice, &obj) != LR_OK) return 2;\n"
+        "  return (choice[0] == 1 && choice[1] == 0 && obj == 8.0) ? 0 : 3;\n"
+        "}\n")
+    libdir = os.path.join(ROOT, "rank_linear_layers_b200")
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-llrlinear",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
