@@ -344,11 +344,40 @@ def single_layer_bench(lr, dev, steps=200, warmup=20):
         def st(i):
             lr.lr_linear(X, A, B, None, Y=Y)
         t = time_steps(st, steps, warmup) / steps
-        return {"us_per_call": t * 1e6, "gpu_launches_per_call": int(per_call),
-                "flops": acc.flops(16, 256, 107, 256),
-                "note": "M=16 K=256 r=107 N=256, decode path, back-to-back calls"}
+        out = {"us_per_call": t * 1e6, "gpu_launches_per_call": int(per_call),
+               "flops": acc.flops(16, 256, 107, 256),
+               "note": "M=16 K=256 r=107 N=256, decode path, back-to-back calls"}
     except Exception as ex:  # pragma: no cover - reported, not hidden
         return {"error": str(ex)[:200]}
+    # The launch floor: the same calls captured in one CUDA graph.  The
+    # library keeps a workspace per stream, so the capture stream is warmed
+    # up first (nothing is allocated while capturing).
+    try:
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            for i in range(3):
+                st(i)
+        cs.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            for i in range(steps):
+                st(i)
+        g.replay()
+        torch.cuda.synchronize()
+        cur = torch.cuda.current_stream()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for _ in range(3):
+            g.replay()
+        e1.record(cur)
+        torch.cuda.synchronize()
+        out["graph_us_per_call"] = e0.elapsed_time(e1) * 1e3 / (3 * steps)
+        del g
+    except Exception as ex:  # pragma: no cover - reported, not hidden
+        out["graph_error"] = str(ex)[:200]
+    return out
 
 
 def misalignment_check(lr, dev, l2, ranks=range(1000, 1009)):
