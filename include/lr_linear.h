@@ -20,7 +20,9 @@
  * Conventions for every entry point:
  *   - All tensors are bf16 (IEEE bfloat16 bit patterns), row-major and
  *     contiguous unless a leading dimension is given.  Accumulation is fp32;
- *     Y is rounded once to bf16 (nearest-even) after the bias is added.
+ *     Y is rounded once to bf16 (nearest-even) after the bias is added, or
+ *     stored unrounded in fp32 by lr_linear_f32 (and by group entries with
+ *     y_f32 set).
  *   - Device pointers point to memory of the current CUDA device.  Any
  *     2-byte-aligned pointer is accepted; 16-byte-aligned pointers with row
  *     strides that are multiples of 8 elements take the TMA fast path.
@@ -82,15 +84,40 @@ typedef enum {
  * A or B of the next call turns the early copy off (lr_set_early_copy).
  * Results are deterministic except that split K (small prefill GEMMs, see
  * lr_set_split_k) adds fp32 partial sums in a run-dependent order.
+ *
+ * Precision of T on the prefill path: the tensor cores take bf16 operands,
+ * so GEMM2 reads T either rounded once to bf16 or as two bf16 parts
+ * hi = bf16(T), lo = bf16(T − hi) multiplied into the same fp32 accumulator
+ * (about 16 significant bits of T; twice GEMM2's tensor work).  The automatic
+ * choice takes the two parts whenever the extra tensor work (2·M·r·N FLOPs)
+ * costs at most a third of the call's ideal time, max(2·M·r·(K+N) FLOPs at
+ * 1.6 PFLOP/s, (MK+Kr+rN+MN)·2 bytes at 6.4 TB/s, 5 µs): small calls, and
+ * bandwidth-bound ones such as small r at large M, K, N.
+ * lr_set_t_precision overrides it.  The decode path keeps T in fp32.
  */
 lr_status lr_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
                     int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
 
 /*
+ * lr_linear_f32 — lr_linear with Y [M,N] written as fp32 (IEEE binary32):
+ * the fp32 accumulator plus bias, without the final rounding to bf16 (Y
+ * 4-byte aligned).  Same kernels, paths and T precision as lr_linear; the
+ * bf16 result of lr_linear is this value rounded to nearest-even whenever
+ * both calls add their partial sums in the same order (no split K).  The
+ * accuracy the methods' pages state (bf16 inputs, fp32 accumulation) is a
+ * property of this value: rounding Y to bf16 adds up to 2^-8·|Y| per
+ * element on top of it.  Not available on the CTA-pair path (path 4:
+ * LR_ERR_UNSUPPORTED).
+ */
+lr_status lr_linear_f32(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                        int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
+
+/*
  * One projection of a group (a decoder layer's q/k/v/o/gate/up/down).
  * X [M,K] (entries may share one X pointer), A [K,r], B [r,N], bias [N] or
  * NULL, Y with row stride ld_y >= N (so two projections can write the two
- * halves of one packed [M, N1+N2] buffer, e.g. gate and up).
+ * halves of one packed [M, N1+N2] buffer, e.g. gate and up).  y_f32 = 0: Y
+ * is bf16; nonzero: Y is fp32 as in lr_linear_f32 (4-byte aligned).
  */
 typedef struct {
   const void* X;
@@ -102,6 +129,7 @@ typedef struct {
   int64_t ld_y;
   int64_t r;
   int64_t N;
+  int32_t y_f32;
 } lr_proj;
 
 /*
@@ -208,13 +236,17 @@ int lr_last_cuda_error(void);
  *   for all earlier work on the stream, so a caller's kernel that starts
  *   its dependents early can safely write the next call's operands.  Other
  *   values return LR_ERR_INVALID_ARG.
- * All five are process-wide and take effect on the next call.
+ * lr_set_t_precision — how a prefill GEMM2 reads T: 0 = automatic (the
+ *   default, see lr_linear), 1 = T rounded once to bf16, 2 = T as two bf16
+ *   parts hi + lo.  Other values return LR_ERR_INVALID_ARG.
+ * All six are process-wide and take effect on the next call.
  */
 lr_status lr_set_path(int path);
 lr_status lr_set_wait_limit_ns(int64_t ns);
 lr_status lr_set_tile_n(int bn);
 lr_status lr_set_split_k(int on);
 lr_status lr_set_early_copy(int on);
+lr_status lr_set_t_precision(int mode);
 
 /*
  * lr_set_withhold_first_stage — testing failure detection only.  With on = 1,

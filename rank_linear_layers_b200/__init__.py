@@ -30,12 +30,15 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_PREFILL_1SM, PATH_PREFILL_PAIR = 0, 1
 
 # Every symbol include/lr_linear.h declares.
 EXPORTS = (
-    "lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense", "lr_last_device_status",
+    "lr_linear", "lr_linear_f32", "lr_linear_group", "lr_linear_host", "lr_dense",
+    "lr_last_device_status",
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
     "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
     "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy",
-    "lr_gac_select",
+    "lr_gac_select", "lr_set_t_precision",
 )
+
+T_AUTO, T_BF16, T_TWO_PARTS = 0, 1, 2
 
 
 class LrError(RuntimeError):
@@ -50,6 +53,7 @@ class LrProj(ctypes.Structure):
         ("X", ctypes.c_void_p), ("K", ctypes.c_int64), ("A", ctypes.c_void_p),
         ("B", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("Y", ctypes.c_void_p),
         ("ld_y", ctypes.c_int64), ("r", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("y_f32", ctypes.c_int32),
     ]
 
 
@@ -68,6 +72,7 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L = ctypes.CDLL(path)
     vp, i64 = ctypes.c_void_p, ctypes.c_int64
     L.lr_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    L.lr_linear_f32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_linear_group.argtypes = [ctypes.POINTER(LrProj), ctypes.c_int, i64, vp]
     L.lr_linear_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_dense.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
@@ -82,17 +87,19 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_set_tile_n.argtypes = [ctypes.c_int]
     L.lr_set_split_k.argtypes = [ctypes.c_int]
     L.lr_set_early_copy.argtypes = [ctypes.c_int]
+    L.lr_set_t_precision.argtypes = [ctypes.c_int]
     ip, lp, dp = (ctypes.POINTER(ctypes.c_int), ctypes.POINTER(i64),
                   ctypes.POINTER(ctypes.c_double))
     L.lr_gac_select.argtypes = [ctypes.c_int, ip, lp, dp, lp, i64, i64, ip, dp]
     L.lr_kernel_launch_count.argtypes = []
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
-    for name in ("lr_linear", "lr_linear_group", "lr_linear_host", "lr_dense",
+    for name in ("lr_linear", "lr_linear_f32", "lr_linear_group", "lr_linear_host", "lr_dense",
                  "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces", "lr_set_withhold_first_stage",
-                 "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy", "lr_gac_select"):
+                 "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy", "lr_gac_select",
+                 "lr_set_t_precision"):
         getattr(L, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = L
@@ -152,6 +159,27 @@ def lr_linear(X, A, B, bias=None, Y=None, stream=None):
     return Y
 
 
+def lr_linear_f32(X, A, B, bias=None, Y=None, stream=None):
+    """Y = (X·A)·B + bias with Y in fp32 (the accumulator plus bias, not
+    rounded to bf16); inputs bf16 as for lr_linear."""
+    import torch
+    M, K = X.shape
+    r = A.shape[1]
+    N = B.shape[1]
+    _check_bf16("X", X)
+    _check_bf16("A", A, (K, r))
+    _check_bf16("B", B, (r, N))
+    _check_bf16("bias", bias, (N,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    if Y.dtype != torch.float32 or not Y.is_cuda or not Y.is_contiguous() or \
+            tuple(Y.shape) != (M, N):
+        raise TypeError("Y must be a contiguous fp32 CUDA tensor of shape (M, N)")
+    _check(lib().lr_linear_f32(_ptr(X), _ptr(A), _ptr(B), _ptr(bias), _ptr(Y), M, K, r, N,
+                               _stream_ptr(stream)), "lr_linear_f32")
+    return Y
+
+
 def lr_dense(X, W, bias=None, Y=None, stream=None):
     """Y = X·W + bias with the same kernels (the dense comparison)."""
     import torch
@@ -173,9 +201,11 @@ def lr_linear_group(projs: Sequence[dict], M: int, stream=None):
 
     Each dict has X, A, B, Y (torch tensors or raw pointer ints), and
     optionally bias, ld_y (default N), K, r, N (taken from shapes when the
-    entries are tensors).  Y may be a view into a packed buffer: pass the
-    element pointer and ld_y explicitly via ``Y_ptr`` / ``ld_y``.
+    entries are tensors) and y_f32 (Y is fp32; default: inferred from a Y
+    tensor's dtype, else bf16).  Y may be a view into a packed buffer: pass
+    the element pointer and ld_y explicitly via ``Y_ptr`` / ``ld_y``.
     """
+    import torch
     arr = (LrProj * max(1, len(projs)))()
     for i, p in enumerate(projs):
         A, B = p["A"], p["B"]
@@ -183,11 +213,12 @@ def lr_linear_group(projs: Sequence[dict], M: int, stream=None):
         r = p.get("r", A.shape[1] if hasattr(A, "shape") else None)
         N = p.get("N", B.shape[1] if hasattr(B, "shape") else None)
         y_ptr = p.get("Y_ptr", _ptr(p.get("Y")))
+        y32 = p.get("y_f32", getattr(p.get("Y"), "dtype", None) == torch.float32)
         arr[i] = LrProj(_ptr(p["X"]) if hasattr(p["X"], "data_ptr") else p["X"], K,
                         _ptr(A) if hasattr(A, "data_ptr") else A,
                         _ptr(B) if hasattr(B, "data_ptr") else B,
                         _ptr(p.get("bias")) if hasattr(p.get("bias"), "data_ptr") else p.get("bias"),
-                        y_ptr, p.get("ld_y", N), r, N)
+                        y_ptr, p.get("ld_y", N), r, N, 1 if y32 else 0)
     _check(lib().lr_linear_group(arr, len(projs), M, _stream_ptr(stream)), "lr_linear_group")
 
 
@@ -229,6 +260,12 @@ def set_split_k(on):
     off, True/1 on (the default), 2 also where the schedule model predicts a
     shorter launch (experimental)."""
     _check(lib().lr_set_split_k(int(on)), "lr_set_split_k")
+
+
+def set_t_precision(mode: int):
+    """How a prefill GEMM2 reads T: T_AUTO (0, the default), T_BF16 (1, T
+    rounded once to bf16) or T_TWO_PARTS (2, T as bf16 hi + lo)."""
+    _check(lib().lr_set_t_precision(int(mode)), "lr_set_t_precision")
 
 
 def set_early_copy(on: bool):

@@ -27,6 +27,7 @@ std::atomic<int> g_withhold{0};
 std::atomic<int> g_tile_n{0};
 std::atomic<int> g_split_k{1};
 std::atomic<int> g_early_copy{1};
+std::atomic<int> g_t_precision{0};
 constexpr long long kDefaultWaitNs = 2000000000LL;
 
 struct DeviceInfo {
@@ -232,7 +233,7 @@ WaitCtl wait_ctl(DeviceInfo* d) {
 }
 
 lr_status validate(const void* X, const void* A, const void* B, const void* bias, const void* Y,
-                   int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy) {
+                   int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, bool y_f32 = false) {
   if (M < 0 || K < 0 || r < 0 || N < 0) return LR_ERR_INVALID_ARG;
   if (M > kMaxDim || K > kMaxDim || r > kMaxDim || N > kMaxDim) return LR_ERR_UNSUPPORTED;
   if (ldy < N) return LR_ERR_INVALID_ARG;
@@ -240,7 +241,8 @@ lr_status validate(const void* X, const void* A, const void* B, const void* bias
   if (M > 0 && K > 0 && r > 0 && N > 0 && (!X || !A || !B)) return LR_ERR_INVALID_ARG;
   for (const void* p : {X, A, B, bias, Y})
     if (p && !aligned2(p)) return LR_ERR_INVALID_ARG;
-  const size_t ybytes = span_bytes(M, N, ldy);
+  if (y_f32 && Y && (reinterpret_cast<uintptr_t>(Y) & 3u) != 0) return LR_ERR_INVALID_ARG;
+  const size_t ybytes = span_bytes(M, N, ldy) * (y_f32 ? 2 : 1);
   if (ranges_overlap(Y, ybytes, X, span_bytes(M, K, K)) ||
       ranges_overlap(Y, ybytes, A, span_bytes(K, r, r)) ||
       ranges_overlap(Y, ybytes, B, span_bytes(r, N, N)) ||
@@ -292,7 +294,7 @@ size_t ctr_bytes(int M, int64_t Kd, int64_t n, int sms) {
 
 lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                      const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
-                     int64_t N, int64_t ldy) {
+                     int64_t N, int64_t ldy, bool y_f32) {
   const int m = static_cast<int>(M);
   const size_t acc1 = acc_bytes(m, r), acc2 = acc_bytes(m, N);
   const size_t c1 = ctr_bytes(m, K, r, d->sms), c2 = ctr_bytes(m, r, N, d->sms);
@@ -311,6 +313,9 @@ lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const vo
   if (st != LR_OK) return st;
   // Phase 2 starts streaming B while phase 1 finishes (programmatic
   // dependent launch); it reads T only after phase 1 has completed.
+  if (y_f32)
+    return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, static_cast<float*>(Y), ldy,
+                  nullptr, 0, bias, true);
   return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias, true);
 }
 
@@ -453,6 +458,7 @@ lr_status chain_problem(ChainBuild& cb, int map_a, int a_col0, int map_b, int64_
   P.Kc = static_cast<int>(Kc);
   P.map_a = map_a;
   P.map_b = map_b;
+  P.map_a_lo = -1;
   P.a_col0 = a_col0;
   P.c = static_cast<__nv_bfloat16*>(c);
   P.ldc = ldc;
@@ -476,6 +482,12 @@ double epilogue_us(int bn) { return 0.6 + 1.0 * bn / 256.0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Simulate the static round-robin schedule of the chain kernel.
+// A k block of a problem whose operand a has two parts issues twice the
+// tensor-core work of its tile width.
+double kblock_cost(const ChainProblem& P, int bn) {
+  return kblock_us(P.map_a_lo >= 0 ? 2 * bn : bn);
+}
+
 double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
   int64_t total = 0;
   for (int i = 0; i < a.n_prob; ++i)
@@ -488,7 +500,7 @@ double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
   for (int i = 0; i < a.n_prob; ++i) {
     const ChainProblem& P = a.p[i];
     const int64_t tm = ceil_div(P.Mr, kGemmBM), tn = ceil_div(P.Nc, bn[i]);
-    const double dur = static_cast<double>(ceil_div(P.Kc, kGemmBK)) * kblock_us(bn[i]) + 0.15;
+    const double dur = static_cast<double>(ceil_div(P.Kc, kGemmBK)) * kblock_cost(P, bn[i]) + 0.15;
     std::vector<double>* sig = nullptr;
     const std::vector<double>* wait = nullptr;
     if (P.signal_group >= 0) {
@@ -550,7 +562,7 @@ double simulate_chain_split(const ChainArgs& a, const std::vector<int>& bn,
         double& tc = t[static_cast<size_t>(idx % G)];
         double start = tc;
         if (wait && m < static_cast<int64_t>(wait->size())) start = std::max(start, (*wait)[m]);
-        tc = start + static_cast<double>(kb) * kblock_us(bn[i]) + 0.15;
+        tc = start + static_cast<double>(kb) * kblock_cost(P, bn[i]) + 0.15;
         if (sig) (*sig)[m] = std::max((*sig)[m], tc + epilogue_us(bn[i]) + fin);
       }
     }
@@ -570,20 +582,22 @@ std::vector<int> plan_chain(const ChainArgs& a, int sms) {
   std::vector<int64_t> key{sms, forced};
   for (int i = 0; i < a.n_prob; ++i) {
     const ChainProblem& P = a.p[i];
-    key.insert(key.end(), {P.Mr, P.Nc, P.Kc, P.wait_group, P.signal_group});
+    key.insert(key.end(), {P.Mr, P.Nc, P.Kc, P.wait_group, P.signal_group, P.map_a_lo >= 0});
   }
   {
     std::lock_guard<std::mutex> lk(g_plan_mu);
     auto it = g_plans.find(key);
     if (it != g_plans.end()) return it->second;
   }
+  // Two-part operand a: both parts and the b tile share a stage (bn <= 128).
+  auto cap = [&](int i) { return a.p[i].map_a_lo >= 0 ? 128 : 256; };
   std::vector<int> bn(static_cast<size_t>(a.n_prob), 256);
   if (forced > 0) {
-    std::fill(bn.begin(), bn.end(), forced);
+    for (int i = 0; i < a.n_prob; ++i) bn[i] = std::min(forced, cap(i));
   } else {
     std::vector<std::vector<int>> cand(static_cast<size_t>(a.n_prob));
     for (int i = 0; i < a.n_prob; ++i) {
-      const int top = static_cast<int>(std::min<int64_t>(256, ceil_div(a.p[i].Nc, 32) * 32));
+      const int top = static_cast<int>(std::min<int64_t>(cap(i), ceil_div(a.p[i].Nc, 32) * 32));
       for (int b = top; b >= 32; b -= 32) cand[i].push_back(b);
       bn[i] = top;
     }
@@ -774,18 +788,49 @@ lr_status tma_operand(DeviceInfo* d, cudaStream_t stream, const void* p, int64_t
   return LR_OK;
 }
 
+// Whether a prefill GEMM2 Y = T·B takes T as two bf16 parts, hi = bf16(T) and
+// lo = bf16(T - hi) (about 16 significant bits, two tensor-core products per
+// k step), instead of T rounded once to bf16.  Rounding T adds an error of
+// relative size about 2^-9/sqrt(3) to every output (on top of the output's
+// own rounding when Y is bf16), whatever the shape; the two parts remove it
+// and add GEMM2's tensor work once more.  Automatic choice
+// (lr_set_t_precision(0)): two parts whenever that extra work costs at most
+// a third of the call's ideal time, max(FLOPs / tensor peak, bytes / HBM
+// bandwidth, 5 µs of launch latency), with B200's dense bf16 peak
+// (1.6 PFLOP/s) and HBM bandwidth (6.4 TB/s) as measured with cuBLAS and a
+// device copy.
+bool t_in_two_parts(int64_t M, int64_t K, int64_t r, int64_t N) {
+  const int mode = g_t_precision.load();
+  if (mode == 1) return false;
+  if (mode == 2) return true;
+  const double peak = 1.6e15, bw = 6.4e12;
+  const double m = static_cast<double>(M), k = static_cast<double>(K),
+               rr = static_cast<double>(r), n = static_cast<double>(N);
+  const double extra = 2.0 * m * rr * n / peak;
+  const double ideal = std::max({2.0 * m * rr * (k + n) / peak,
+                                 2.0 * (m * k + k * rr + rr * n + m * n) / bw, 5e-6});
+  return 3.0 * extra <= ideal;
+}
+
 lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                       const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
-                      int64_t N, int64_t ldy) {
+                      int64_t N, int64_t ldy, bool y_f32) {
   const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), kPitchElems));
   const size_t tbytes = align_up(static_cast<size_t>(M) * ldt * 2, 256);
   const size_t rp = repack_bytes(X, K, M, K) + repack_bytes(A, r, K, r) + repack_bytes(B, N, r, N);
   const bool pairs = g_path.load() == 4;
+  if (pairs && y_f32) return LR_ERR_UNSUPPORTED;
+  const bool two = !pairs && t_in_two_parts(M, K, r, N);
   char *zero = nullptr, *scratch = nullptr;
-  lr_status st = workspace(stream, 0, tbytes + (pairs ? rp : 0), &zero, &scratch);
+  lr_status st = workspace(stream, 0, tbytes * (two ? 2 : 1) + (pairs ? rp : 0), &zero, &scratch);
   if (st != LR_OK) return st;
   void* T = scratch;
   scratch += tbytes;
+  __nv_bfloat16* T_lo = nullptr;
+  if (two) {
+    T_lo = reinterpret_cast<__nv_bfloat16*>(scratch);
+    scratch += tbytes;
+  }
   // Misaligned operands are realigned into an area of their own; the
   // call's first repack may overlap the previous launch (see repack_area).
   bool early = false;
@@ -816,10 +861,11 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   const bool after_repack = repacks > 0;
   auto dep = [&](const void* used, const void* given) { return !after_repack || used != given; };
   ChainBuild cb;
-  int mx, ma, mt, mb;
+  int mx, ma, mt, mb, mt_lo = -1;
   if ((st = chain_map(cb, x.p, K, M, x.ld, true, &mx)) != LR_OK) return st;
   if ((st = chain_map(cb, a.p, r, K, a.ld, false, &ma)) != LR_OK) return st;
   if ((st = chain_map(cb, T, r, M, ldt, true, &mt)) != LR_OK) return st;
+  if (two && (st = chain_map(cb, T_lo, r, M, ldt, true, &mt_lo)) != LR_OK) return st;
   if ((st = chain_map(cb, b.p, N, r, b.ld, false, &mb)) != LR_OK) return st;
   // GEMM1's columns: when whole 256-column tiles already take more than one
   // wave and the last tile would be at most half full, the tail columns are
@@ -831,22 +877,30 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
     st = chain_problem(cb, mx, 0, ma, M, main_cols, K, T, ldt, nullptr, -1, 0, dep(x.p, X),
                        dep(a.p, A));
     if (st != LR_OK) return st;
+    cb.args.p[cb.args.n_prob - 1].c_lo = T_lo;
     st = chain_problem(cb, mx, 0, ma, M, tail, K, static_cast<__nv_bfloat16*>(T) + main_cols, ldt,
                        nullptr, -1, 0, dep(x.p, X), dep(a.p, A), static_cast<int>(main_cols));
+    if (st != LR_OK) return st;
+    cb.args.p[cb.args.n_prob - 1].c_lo = two ? T_lo + main_cols : nullptr;
   } else {
     st = chain_problem(cb, mx, 0, ma, M, r, K, T, ldt, nullptr, -1, 0, dep(x.p, X), dep(a.p, A));
+    if (st != LR_OK) return st;
+    cb.args.p[cb.args.n_prob - 1].c_lo = T_lo;
   }
-  if (st != LR_OK) return st;
   st = chain_problem(cb, mt, 0, mb, M, N, r, Y, ldy, bias, 0, -1, false, dep(b.p, B));
   if (st != LR_OK) return st;
+  cb.args.p[cb.args.n_prob - 1].map_a_lo = mt_lo;
+  if (y_f32) cb.args.p[cb.args.n_prob - 1].c32 = static_cast<float*>(Y);
   st = run_chain(d, stream, cb);
-  note_call(stream, st == LR_OK, Y, span_bytes(M, N, ldy), cb.args.total_tiles >= d->sms);
+  note_call(stream, st == LR_OK, Y, span_bytes(M, N, ldy) * (y_f32 ? 2 : 1),
+            cb.args.total_tiles >= d->sms);
   return st;
 }
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
-                     int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, cudaStream_t stream) {
-  lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy);
+                     int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, cudaStream_t stream,
+                     bool y_f32 = false) {
+  lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
   if (st != LR_OK) return st;
   const int path = g_path.load();
   if (path == 1 && M > 16) return LR_ERR_INVALID_ARG;
@@ -855,17 +909,18 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
   int dev = 0;
   st = device_info(&d, &dev);
   if (st != LR_OK) return st;
+  const size_t ybytes = span_bytes(M, N, ldy) * (y_f32 ? 2 : 1);
   if (K == 0 || r == 0) {
-    note_call(stream, false, Y, span_bytes(M, N, ldy));
-    return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), ldy, M, N,
-                                     static_cast<const __nv_bfloat16*>(bias), stream));
+    note_call(stream, false, Y, ybytes);
+    return launched(launch_fill_bias(Y, y_f32, ldy, M, N, static_cast<const __nv_bfloat16*>(bias),
+                                     stream));
   }
   const bool decode = (path == 1) || (path == 0 && M <= 16);
   if (decode) {
-    note_call(stream, false, Y, span_bytes(M, N, ldy));
-    return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+    note_call(stream, false, Y, ybytes);
+    return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
   }
-  return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy);
+  return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
 }
 
 
@@ -881,7 +936,9 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
 // launch) when the group does not fit one launch's tables.
 lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* projs, int n,
                             int64_t M) {
-  for (int i = 0; i < n; ++i) note_call(stream, false, projs[i].Y, span_bytes(M, projs[i].N, projs[i].ld_y));
+  for (int i = 0; i < n; ++i)
+    note_call(stream, false, projs[i].Y,
+              span_bytes(M, projs[i].N, projs[i].ld_y) * (projs[i].y_f32 ? 2 : 1));
   struct Set {
     const void* X;
     int64_t K;
@@ -889,6 +946,7 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
     int64_t width = 0;  // columns of T_set (sum of slices)
     int64_t pitch = 0;  // row pitch of T_set and A_set: width in 128-byte rows
     bool concat = false;  // A copied into a concatenated factor
+    bool two = false;     // T_set also written as a low part (some member reads two parts)
   };
   std::vector<Set> sets;
   std::vector<int64_t> off(static_cast<size_t>(n), 0);
@@ -901,26 +959,31 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
     for (size_t k = 0; k < sets.size(); ++k)
       if (sets[k].X == p.X && sets[k].K == p.K) si = static_cast<int>(k);
     if (si < 0) {
-      sets.push_back(Set{p.X, p.K, {}, 0, false});
+      sets.push_back(Set{p.X, p.K, {}, 0, 0, false, false});
       si = static_cast<int>(sets.size()) - 1;
     }
     Set& st = sets[static_cast<size_t>(si)];
     off[static_cast<size_t>(i)] = st.width;
     st.width += static_cast<int64_t>(align_up(static_cast<size_t>(p.r), 8));
     st.members.push_back(i);
+    if (t_in_two_parts(M, p.K, p.r, p.N)) st.two = true;
     set_of[static_cast<size_t>(i)] = si;
     ++gemm2;
   }
-  for (Set& st : sets) st.pitch = static_cast<int64_t>(align_up(static_cast<size_t>(st.width), kPitchElems));
+  int n_two = 0;
+  for (Set& st : sets) {
+    st.pitch = static_cast<int64_t>(align_up(static_cast<size_t>(st.width), kPitchElems));
+    n_two += st.two ? 1 : 0;
+  }
   if (static_cast<int>(sets.size()) + gemm2 > kChainMaxProbs ||
-      3 * static_cast<int>(sets.size()) + gemm2 > kChainMaxMaps)
+      3 * static_cast<int>(sets.size()) + n_two + gemm2 > kChainMaxMaps)
     return LR_ERR_UNSUPPORTED;
   // Workspace: T per set, concatenated factors, realigned X and B copies.
   size_t need = 0;
   for (Set& st : sets) {
     const lr_proj& p0 = projs[st.members[0]];
     st.concat = st.members.size() > 1 || !tma_ok(p0.A, p0.r);
-    need += align_up(static_cast<size_t>(M) * st.pitch * 2, 256);
+    need += align_up(static_cast<size_t>(M) * st.pitch * 2, 256) * (st.two ? 2 : 1);
     if (st.concat) need += align_up(static_cast<size_t>(st.K) * st.pitch * 2, 256);
     need += repack_bytes(st.X, st.K, M, st.K);
   }
@@ -933,7 +996,7 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
   for (int i = 0; i < n; ++i) {
     const lr_proj& p = projs[i];
     if (M > 0 && p.N > 0 && (p.K == 0 || p.r == 0)) {
-      stt = launched(launch_fill_bias(static_cast<__nv_bfloat16*>(p.Y), p.ld_y, M, p.N,
+      stt = launched(launch_fill_bias(p.Y, p.y_f32 != 0, p.ld_y, M, p.N,
                                       static_cast<const __nv_bfloat16*>(p.bias), stream));
       if (stt != LR_OK) return stt;
     }
@@ -942,6 +1005,7 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
   int repacks = 0;
   struct SetOps {
     void* T;
+    __nv_bfloat16* T_lo;
     Operand x, a;
   };
   std::vector<SetOps> ops(sets.size());
@@ -949,6 +1013,11 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
     Set& st = sets[k];
     ops[k].T = scratch;
     scratch += align_up(static_cast<size_t>(M) * st.pitch * 2, 256);
+    ops[k].T_lo = nullptr;
+    if (st.two) {
+      ops[k].T_lo = reinterpret_cast<__nv_bfloat16*>(scratch);
+      scratch += align_up(static_cast<size_t>(M) * st.pitch * 2, 256);
+    }
     stt = tma_operand(d, stream, st.X, st.K, M, st.K, &scratch, &ops[k].x, &repacks);
     if (stt != LR_OK) return stt;
     if (st.concat) {
@@ -979,7 +1048,7 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
   const bool after_repack = repacks > 0;
   auto dep = [&](const void* used, const void* given) { return !after_repack || used != given; };
   ChainBuild cb;
-  std::vector<int> tmap(sets.size());
+  std::vector<int> tmap(sets.size()), tmap_lo(sets.size(), -1);
   for (size_t k = 0; k < sets.size(); ++k) {
     const Set& st = sets[k];
     const lr_proj& p0 = projs[st.members[0]];
@@ -991,9 +1060,13 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
     // zero); a concatenated T's slice pads are written as zero by GEMM1.
     if ((stt = chain_map(cb, ops[k].T, nc, M, st.pitch, true, &mt)) != LR_OK) return stt;
     tmap[k] = mt;
+    if (st.two &&
+        (stt = chain_map(cb, ops[k].T_lo, nc, M, st.pitch, true, &tmap_lo[k])) != LR_OK)
+      return stt;
     stt = chain_problem(cb, mx, 0, ma, M, nc, st.K, ops[k].T, st.pitch, nullptr, -1,
                         static_cast<int>(k), dep(ops[k].x.p, st.X), dep(ops[k].a.p, p0.A));
     if (stt != LR_OK) return stt;
+    cb.args.p[cb.args.n_prob - 1].c_lo = ops[k].T_lo;
   }
   for (size_t k = 0; k < sets.size(); ++k) {
     for (int i : sets[k].members) {
@@ -1004,6 +1077,9 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
       stt = chain_problem(cb, tmap[k], static_cast<int>(off[static_cast<size_t>(i)]), mb, M, p.N,
                           p.r, p.Y, p.ld_y, p.bias, static_cast<int>(k), -1, false, dep(b.p, p.B));
       if (stt != LR_OK) return stt;
+      ChainProblem& P = cb.args.p[cb.args.n_prob - 1];
+      if (t_in_two_parts(M, p.K, p.r, p.N)) P.map_a_lo = tmap_lo[k];
+      if (p.y_f32) P.c32 = static_cast<float*>(p.Y);
     }
   }
   return run_chain(d, stream, cb);
@@ -1015,12 +1091,14 @@ lr_status run_group_prefill(DeviceInfo* d, cudaStream_t stream, const lr_proj* p
 // ranges overlap at all.
 bool y_disjoint(const lr_proj& p, const lr_proj& q, int64_t M) {
   if (!p.Y || !q.Y || M == 0 || p.N == 0 || q.N == 0) return true;
-  if (!ranges_overlap(p.Y, span_bytes(M, p.N, p.ld_y), q.Y, span_bytes(M, q.N, q.ld_y)))
+  const int64_t es = p.y_f32 ? 4 : 2;
+  if (!ranges_overlap(p.Y, span_bytes(M, p.N, p.ld_y) * (es / 2), q.Y,
+                      span_bytes(M, q.N, q.ld_y) * (q.y_f32 ? 2 : 1)))
     return true;
-  if (p.ld_y != q.ld_y) return false;
+  if (p.ld_y != q.ld_y || (p.y_f32 != 0) != (q.y_f32 != 0)) return false;
   const intptr_t d = reinterpret_cast<intptr_t>(q.Y) - reinterpret_cast<intptr_t>(p.Y);
-  if (d % 2 != 0) return false;
-  const int64_t off = d / 2, ld = p.ld_y;
+  if (d % es != 0) return false;
+  const int64_t off = d / es, ld = p.ld_y;
   int64_t a = off / ld, b = off % ld;
   if (b < 0) {
     b += ld;
@@ -1066,14 +1144,19 @@ lr_status lr_linear(const void* X, const void* A, const void* B, const void* bia
   return run_linear(X, A, B, bias, Y, M, K, r, N, N, static_cast<cudaStream_t>(stream));
 }
 
+lr_status lr_linear_f32(const void* X, const void* A, const void* B, const void* bias, void* Y,
+                        int64_t M, int64_t K, int64_t r, int64_t N, void* stream) {
+  return run_linear(X, A, B, bias, Y, M, K, r, N, N, static_cast<cudaStream_t>(stream), true);
+}
+
 lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream) {
   if (n_proj < 0 || (n_proj > 0 && !projs) || M < 0) return LR_ERR_INVALID_ARG;
   // Validate everything before the first launch, including Y overlaps.
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];
-    lr_status st = validate(p.X, p.A, p.B, p.bias, p.Y, M, p.K, p.r, p.N, p.ld_y);
+    lr_status st = validate(p.X, p.A, p.B, p.bias, p.Y, M, p.K, p.r, p.N, p.ld_y, p.y_f32 != 0);
     if (st != LR_OK) return st;
-    const size_t yi = span_bytes(M, p.N, p.ld_y);
+    const size_t yi = span_bytes(M, p.N, p.ld_y) * (p.y_f32 ? 2 : 1);
     for (int j = 0; j < n_proj; ++j) {
       const lr_proj& q = projs[j];
       if (j != i) {
@@ -1099,7 +1182,7 @@ lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* str
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];
     lr_status st = run_linear(p.X, p.A, p.B, p.bias, p.Y, M, p.K, p.r, p.N, p.ld_y,
-                              static_cast<cudaStream_t>(stream));
+                              static_cast<cudaStream_t>(stream), p.y_f32 != 0);
     if (st != LR_OK) return st;
   }
   return LR_OK;
@@ -1166,8 +1249,8 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
   st = device_info(&d, &dev);
   if (st != LR_OK) return st;
   if (K == 0)
-    return launched(launch_fill_bias(static_cast<__nv_bfloat16*>(Y), N, M, N,
-                                     static_cast<const __nv_bfloat16*>(bias), stream));
+    return launched(launch_fill_bias(Y, false, N, M, N, static_cast<const __nv_bfloat16*>(bias),
+                                     stream));
   const int path = g_path.load();
   const bool decode = (path == 1) || (path == 0 && M <= 16);
   if (decode) {
@@ -1269,6 +1352,12 @@ lr_status lr_set_split_k(int on) {
 lr_status lr_set_early_copy(int on) {
   if (on != 0 && on != 1) return LR_ERR_INVALID_ARG;
   g_early_copy.store(on);
+  return LR_OK;
+}
+
+lr_status lr_set_t_precision(int mode) {
+  if (mode < 0 || mode > 2) return LR_ERR_INVALID_ARG;
+  g_t_precision.store(mode);
   return LR_OK;
 }
 

@@ -104,12 +104,11 @@ __device__ __forceinline__ void reduce_and_finalise(const SkinnyArgs& a, const f
     float* src = a.acc + static_cast<int64_t>(m) * a.ld_acc + n0 + c;
     const float v = __ldcg(src);
     __stcg(src, 0.f);
-    if (a.out_f32) {
-      a.out_f32[static_cast<int64_t>(m) * a.ld_out_f32 + n0 + c] = v;
-    } else {
-      const float b = a.bias ? __bfloat162float(a.bias[n0 + c]) : 0.f;
+    const float b = a.bias ? __bfloat162float(a.bias[n0 + c]) : 0.f;
+    if (a.out_f32)
+      a.out_f32[static_cast<int64_t>(m) * a.ld_out_f32 + n0 + c] = v + b;
+    else
       a.out_bf16[static_cast<int64_t>(m) * a.ld_out + n0 + c] = __float2bfloat16_rn(v + b);
-    }
   }
   if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
 }

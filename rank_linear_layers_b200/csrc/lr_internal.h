@@ -45,7 +45,7 @@ struct SkinnyArgs {
   unsigned int* counters;  // one per column block, zero at rest
   int k_chunk;             // rows of W per CTA
   int splits;              // == gridDim.y
-  float* out_f32;          // if non-null: fp32 result [M, ld_out_f32]
+  float* out_f32;          // if non-null: fp32 result (+bias) [M, ld_out_f32]
   int64_t ld_out_f32;
   __nv_bfloat16* out_bf16;  // else bf16 result (+bias) [M, ld_out]
   int64_t ld_out;
@@ -141,6 +141,18 @@ struct ChainProblem {
   __nv_bfloat16* c;
   int64_t ldc;
   const __nv_bfloat16* bias;
+  // fp32 output: when c32 is set the result (+bias) is stored unrounded as
+  // fp32 at c32 [Mr, ldc] and c is unused.
+  float* c32;
+  // Two-part output (GEMM1 writing T): when c_lo is set, c receives
+  // hi = bf16(v) and c_lo [Mr, ldc] receives lo = bf16(v - hi), so that
+  // hi + lo carries v to about 16 significant bits.
+  __nv_bfloat16* c_lo;
+  // Two-part operand a (GEMM2 reading T): when map_a_lo >= 0, every k step
+  // is multiplied twice into the same accumulator, once with operand a from
+  // map_a and once from map_a_lo (same coordinates).  Both parts and the
+  // operand-b tile share one pipeline stage, so bn is at most 128.
+  int map_a_lo;
   int wait_group;    // -1, or the counter group that gates operand a
   int wait_count;    // arrivals that complete one row block of that group
   int signal_group;  // -1, or the counter group this problem arrives on
@@ -197,8 +209,9 @@ cudaError_t launch_repack(const __nv_bfloat16* src, int64_t lds, size_t src_byte
                           int num_sms, cudaStream_t stream, bool dependent, WaitCtl wait,
                           bool read_early = false);
 
-// Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0).
-cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+// Y[m, n] = bias[n] (or 0) for an empty contraction (K == 0 or r == 0); Y is
+// bf16, or fp32 when y_f32.
+cudaError_t launch_fill_bias(void* Y, bool y_f32, int64_t ldy, int64_t M, int64_t N,
                              const __nv_bfloat16* bias, cudaStream_t stream);
 
 }  // namespace lr

@@ -127,7 +127,7 @@ extern "C" lr_status lr_linear_decode_static(const void* X, const void* A, const
   lr_status st = static_setup(&scratch, &sms);
   if (st != LR_OK) return st;
   if (K == 0 || r == 0) {
-    cudaError_t e = launch_fill_bias(static_cast<__nv_bfloat16*>(Y), N, M, N,
+    cudaError_t e = launch_fill_bias(Y, false, N, M, N,
                                      static_cast<const __nv_bfloat16*>(bias), stream);
     if (e != cudaSuccess) return fail(e);
     note_launches(1);

@@ -9,10 +9,10 @@
 // layouts from shared memory directly, so no operand is transposed.
 //
 // umma_chain_kernel runs a list of such GEMMs in one persistent launch (one
-// CTA per SM, warp-specialised, 192 threads):
-//   warps 0-3  epilogue: TMEM -> registers -> +bias -> bf16 -> global
-//   warp 4     one elected thread issues tcgen05.mma (128 × bn × 16 per issue)
-//   warp 5     one thread issues the TMA tile loads (128-byte swizzle)
+// CTA per SM, warp-specialised, 320 threads):
+//   warps 0-7  epilogue: TMEM -> registers -> +bias -> bf16 (or fp32) -> global
+//   warp 8     one elected thread issues tcgen05.mma (128 × bn × 16 per issue)
+//   warp 9     one thread issues the TMA tile loads (128-byte swizzle)
 // A 4-stage shared-memory ring (mbarrier full/empty pairs) feeds the MMA;
 // two TMEM accumulators (2 × 256 fp32 columns) let the epilogue of one tile
 // overlap the main loop of the next.  Each problem has its own tile width
@@ -181,6 +181,70 @@ __device__ __forceinline__ void split_add_chunk(uint8_t* buf, const uint32_t (&v
   __syncwarp();
 }
 
+// fp32 output: one 32-row × 32-column chunk (one row per lane) plus bias,
+// unrounded, transposed through the warp's 4 KB buffer (128-byte rows,
+// 16-byte chunks swizzled by row) so that each store covers 4 rows × 128
+// contiguous bytes.
+__device__ __forceinline__ void emit_chunk_f32(uint8_t* buf, const uint32_t (&v)[32], float* c,
+                                               int64_t ldc, const __nv_bfloat16* bias, int row0,
+                                               int Mr, int col0, int cend, bool vec_ok, int lane) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    f[i] = __uint_as_float(v[i]);
+    if (bias && col0 + i < cend) f[i] += __bfloat162float(bias[col0 + i]);
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+        make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+  __syncwarp();
+  const int cq = lane & 7;
+  const int col = col0 + 4 * cq;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int r = 4 * s + (lane >> 3);
+    const float4 u = *reinterpret_cast<const float4*>(buf + r * 128 + ((cq ^ (r & 7)) << 4));
+    const int row = row0 + r;
+    if (row >= Mr || col >= cend) continue;
+    float* dst = c + static_cast<int64_t>(row) * ldc + col;
+    if (vec_ok && col + 4 <= cend) {
+      *reinterpret_cast<float4*>(dst) = u;
+    } else {
+      const float e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (col + i < cend) dst[i] = e[i];
+    }
+  }
+  __syncwarp();
+}
+
+// Store one accumulator chunk in the problem's output form: bf16 (+bias),
+// fp32 (+bias), or the two bf16 parts hi = bf16(v), lo = bf16(v - hi) (no
+// bias).  Uses the warp's whole 4 KB buffer.
+__device__ __forceinline__ void emit_out(const ChainProblem& P, uint8_t* bufs,
+                                         const uint32_t (&v)[32], int row0, int col0, int cend,
+                                         int lane) {
+  if (P.c32) {
+    const bool vec32 = ((reinterpret_cast<uintptr_t>(P.c32) & 15u) == 0) && ((P.ldc & 3) == 0);
+    emit_chunk_f32(bufs, v, P.c32, P.ldc, P.bias, row0, P.Mr, col0, cend, vec32, lane);
+    return;
+  }
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(P.c) & 15u) == 0) && ((P.ldc & 7) == 0);
+  emit_chunk(bufs, v, P.c, P.ldc, P.bias, row0, P.Mr, col0, cend, vec_ok, lane);
+  if (P.c_lo) {
+    uint32_t lo[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float f = __uint_as_float(v[i]);
+      lo[i] = __float_as_uint(f - __bfloat162float(__float2bfloat16_rn(f)));
+    }
+    const bool vec_lo = ((reinterpret_cast<uintptr_t>(P.c_lo) & 15u) == 0) && ((P.ldc & 7) == 0);
+    emit_chunk(bufs + EPI_BOX, lo, P.c_lo, P.ldc, nullptr, row0, P.Mr, col0, cend, vec_lo, lane);
+  }
+}
+
 constexpr int kGemmThreads = 6 * 32;
 
 __device__ __forceinline__ int find_problem(const ChainArgs& g, int tile) {
@@ -274,11 +338,15 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         const int m_blk = otile / P.tiles_n, n_blk = otile - m_blk * P.tiles_n;
         const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
         const int nbox = (P.bn + 63) / 64;
-        const uint32_t bytes = A_STAGE + nbox * B_ATOM;
+        const bool two = P.map_a_lo >= 0;  // bn <= 128: the low part goes after the b tile
+        const uint32_t bytes = (two ? 2 : 1) * A_STAGE + nbox * B_ATOM;
         const CUtensorMap* ma = &maps.m[P.map_a];
+        const CUtensorMap* ma_lo = two ? &maps.m[P.map_a_lo] : nullptr;
         const CUtensorMap* mb = &maps.m[P.map_b];
         auto load_a = [&](int st, int kb) {
-          tma_load_2d(stage_a(st), ma, &full[st], P.a_col0 + (kbase + kb) * BK, m_blk * BM);
+          const int x = P.a_col0 + (kbase + kb) * BK, y = m_blk * BM;
+          tma_load_2d(stage_a(st), ma, &full[st], x, y);
+          if (two) tma_load_2d(stage_b(st) + 2 * B_ATOM, ma_lo, &full[st], x, y);
         };
         auto load_b = [&](int st, int kb) {
           for (int c = 0; c < nbox; ++c)
@@ -368,6 +436,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       const int kbase = (local - (local / P.splits) * P.splits) * P.kb_per_split;
       const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
       const uint32_t idesc = idesc_bf16_f32(BM, P.bn, false, true);
+      const bool two = P.map_a_lo >= 0;
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
       if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait, kWhereMmaAcc)) {
@@ -391,6 +460,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b0 + kk * 2048, B_ATOM, 1024);
             umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (two) {
+              const uint64_t ad_lo = sdesc_sw128(b0 + 2 * B_ATOM + kk * 32, 16, 1024);
+              umma_bf16(d_tmem, ad_lo, bd, idesc, 1u);
+            }
           }
           umma_commit(&empty[s]);
         }
@@ -438,7 +511,14 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       const int nch = (min(P.bn, cend - n0) + 31) / 32;
       uint32_t va[32], vb[32];
       bool last = true;  // this warp's region of the output tile is final
-      if (P.splits == 1) {
+      if (P.splits == 1 && (P.c32 || P.c_lo)) {
+#pragma unroll 1
+        for (int c = half; c < nch; c += 2) {
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), va);
+          tmem_ld_wait(va);
+          emit_out(P, bufs, va, row0, n0 + c * 32, cend, lane);
+        }
+      } else if (P.splits == 1) {
         if (half < nch) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(half * 32), va);
 #pragma unroll 1
         for (int c = half; c < nch; c += 4) {
@@ -485,7 +565,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
               va[4 * q + 3] = __float_as_uint(f.w);
               __stcg(src + q, make_float4(0.f, 0.f, 0.f, 0.f));
             }
-            emit_chunk(bufs, va, P.c, P.ldc, P.bias, row0, P.Mr, n0 + c * 32, cend, vec_ok, lane);
+            emit_out(P, bufs, va, row0, n0 + c * 32, cend, lane);
           }
         }
       }
@@ -719,13 +799,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-__global__ void fill_bias_kernel(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+__global__ void fill_bias_kernel(__nv_bfloat16* Y, float* Y32, int64_t ldy, int64_t M, int64_t N,
                                  const __nv_bfloat16* bias) {
   const int64_t total = M * N;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / N, n = i % N;
-    Y[m * ldy + n] = bias ? bias[n] : __float2bfloat16_rn(0.f);
+    if (Y32)
+      Y32[m * ldy + n] = bias ? __bfloat162float(bias[n]) : 0.f;
+    else
+      Y[m * ldy + n] = bias ? bias[n] : __float2bfloat16_rn(0.f);
   }
 }
 
@@ -772,12 +855,14 @@ cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid,
   return cudaLaunchKernelEx(&cfg, umma_chain_kernel, maps, g);
 }
 
-cudaError_t launch_fill_bias(__nv_bfloat16* Y, int64_t ldy, int64_t M, int64_t N,
+cudaError_t launch_fill_bias(void* Y, bool y_f32, int64_t ldy, int64_t M, int64_t N,
                              const __nv_bfloat16* bias, cudaStream_t stream) {
   const int64_t total = M * N;
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 4096));
-  fill_bias_kernel<<<std::max(blocks, 1), threads, 0, stream>>>(Y, ldy, M, N, bias);
+  fill_bias_kernel<<<std::max(blocks, 1), threads, 0, stream>>>(
+      y_f32 ? nullptr : static_cast<__nv_bfloat16*>(Y), y_f32 ? static_cast<float*>(Y) : nullptr,
+      ldy, M, N, bias);
   return cudaGetLastError();
 }
 

@@ -1,9 +1,15 @@
 """Shared helpers for the GPU parity tests: move generator bits to the GPU,
 read results back, and compare with the oracle at the stated tolerance.
 
-Tolerance (bf16 inputs, fp32 accumulation, bf16 output):
+Tolerance (bf16 inputs, fp32 accumulation), on every compared output:
     max |Y_gpu - Y_ref| <= 2e-2 · RMS(Y_ref)
     ||Y_gpu - Y_ref||_F / ||Y_ref||_F <= 5e-3
+Y_gpu is the library's fp32 output (lr_linear_f32) or its bf16 output.  A
+bf16 output carries one more rounding, up to 2^-8·|Y| per element; where
+even the exact result rounded once to bf16 breaks the bar (the prefill
+q_proj workload: its largest output is 6.7·RMS), the tests check the fp32
+output against the oracle and the bf16 output for equality with that fp32
+output rounded to nearest-even.
 """
 import numpy as np
 
@@ -44,47 +50,15 @@ def compare(Y, Yref, what=""):
     return mx, rel
 
 
-def _bf16_round(x):
-    """Round-to-nearest-even into bf16, returned as float64 (exact)."""
+def rn_bf16(Y32):
+    """fp32 values (numpy or torch) rounded to nearest-even bf16, as float64
+    (torch's conversion): what the library's bf16 output must equal when it
+    is the same fp32 accumulator rounded once."""
     import torch
-    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+    t = Y32 if isinstance(Y32, torch.Tensor) else torch.from_numpy(np.asarray(Y32, np.float32))
+    return t.detach().cpu().float().to(torch.bfloat16).double().numpy()
 
 
-def compare_prefill(Y, p, rows=None, what=""):
-    """The parity bar for the prefill path, with one documented allowance.
-
-    The prefill path rounds T = X·A to bf16 once before the second
-    contraction (the tensor cores take bf16 operands) and Y to bf16 at the
-    end.  On small random shapes those two roundings alone can put the
-    largest element error just past 2e-2·RMS.  When the bar fails, the case
-    passes only if (a) the same arithmetic done on the CPU — fp32 products,
-    T rounded to bf16, fp32 second contraction, bias, Y rounded to bf16 —
-    fails the bar too, by at least as much, and (b) the GPU output agrees
-    with that CPU result element by element within what the two computations
-    may legitimately differ by: one bf16 rounding of Y (2^-7·|Y|) plus one
-    bf16 rounding step of each element of T, whose fp32 sums are formed in
-    different orders (2^-8·(|T|·|B|)).  A wrong kernel fails (b)."""
-    import oracle
-    Yref = oracle.lr_linear(p["X"], p["A"], p["B"], p.get("bias"), rows=rows)
-    try:
-        return compare(Y, Yref, what)
-    except AssertionError:
-        X = lrgen.bf16_to_f64(p["X"])
-        if rows is not None:
-            X = X[rows]
-        A, B = lrgen.bf16_to_f64(p["A"]), lrgen.bf16_to_f64(p["B"])
-        T = _bf16_round((X.astype(np.float32) @ A.astype(np.float32)).astype(np.float64))
-        Z = (T.astype(np.float32) @ B.astype(np.float32)).astype(np.float64)
-        if p.get("bias") is not None:
-            Z = Z + lrgen.bf16_to_f64(p["bias"])
-        E = _bf16_round(Z)
-        S = np.abs(T) @ np.abs(B)
-        rms = float(np.sqrt(np.mean(Yref ** 2)))
-        e_gpu = float(np.abs(np.asarray(Y) - Yref).max()) / rms
-        e_cpu = float(np.abs(E - Yref).max()) / rms
-        assert e_cpu > MAX_ERR_RMS and e_gpu <= e_cpu * 1.05, \
-            f"{what}: GPU max|err| {e_gpu:.3e}·RMS, same roundings on the CPU {e_cpu:.3e}·RMS"
-        allowed = 2.0 ** -7 * np.abs(E) + 2.0 ** -8 * S
-        assert np.all(np.abs(np.asarray(Y) - E) <= allowed), \
-            f"{what}: GPU differs from the CPU rounding model beyond one rounding of Y and of T"
-        return e_gpu, None
+def f32_host(Y32):
+    """A device fp32 tensor as float64 numpy (exact)."""
+    return Y32.detach().cpu().double().numpy()

@@ -12,7 +12,8 @@ import numpy as np
 import pytest
 
 import lrgen
-from helpers import compare_prefill, to_dev, to_f64
+import oracle
+from helpers import compare, f32_host, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -63,7 +64,11 @@ def test_queued_prefill_calls_match_one_at_a_time(lr):
     calls = [(to_dev(q["X"]), to_dev(q["A"]), to_dev(q["B"])) for q in probs]
     ref = one_at_a_time(lr, calls)
     rows = sampled_rows(M, 1)
-    compare_prefill(to_f64(ref[1])[rows], probs[1], rows=rows, what="r=333 sampled rows")
+    q = probs[1]
+    Y32 = lr.lr_linear_f32(*calls[1])
+    torch.cuda.synchronize()
+    compare(f32_host(Y32)[rows], oracle.lr_linear(q["X"], q["A"], q["B"], None, rows=rows),
+            "r=333 sampled rows (fp32 output of the same call)")
     for rep in range(2):
         got = queued(lr, calls)
         for i, (g, e) in enumerate(zip(got, ref)):
@@ -85,7 +90,10 @@ def test_queued_call_reads_previous_output(lr):
     torch.cuda.synchronize()
     assert lr.last_device_status() == lr.LR_OK
     rows = sampled_rows(4096, 2)
-    compare_prefill(to_f64(Y1s)[rows], p1, rows=rows, what="call 1 sampled rows")
+    Y32 = lr.lr_linear_f32(X1, A1, B1)
+    torch.cuda.synchronize()
+    compare(f32_host(Y32)[rows], oracle.lr_linear(p1["X"], p1["A"], p1["B"], None, rows=rows),
+            "call 1 sampled rows (fp32 output of the same call)")
     for rep in range(3):
         Y1 = lr.lr_linear(X1, A1, B1)
         Y2 = lr.lr_linear(X2, Y1, B2)
