@@ -225,11 +225,7 @@ int lr_last_cuda_error(void);
  *   than half the SMs and at least 16 k blocks of 64 (GEMM1 at small ranks)
  *   splits its K loop over several CTAs, which add fp32 partial sums into a
  *   workspace; the last one rounds and stores.  on = 0 turns it off (for
- *   tests and tuning).  on = 2 (experimental) does what 1 does and also
- *   splits the K loop of a launch's GEMM1 2..4 ways when the library's
- *   schedule model (per-k-block and per-epilogue costs, GEMM2's waits on
- *   GEMM1's row blocks) predicts a launch at least 2% shorter.  Other values
- *   return LR_ERR_INVALID_ARG.
+ *   tests and tuning).  Other values return LR_ERR_INVALID_ARG.
  * lr_set_early_copy — on = 1 (the default): a prefill call's realignment
  *   copy may overlap the library's previous prefill launch on the stream
  *   (conditions under lr_linear).  on = 0: every call's first copy waits

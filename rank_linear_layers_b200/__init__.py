@@ -256,10 +256,9 @@ def set_tile_n(bn: int):
 
 
 def set_split_k(on):
-    """Split long K loops of small prefill GEMMs over several CTAs: False/0
-    off, True/1 on (the default), 2 also where the schedule model predicts a
-    shorter launch (experimental)."""
-    _check(lib().lr_set_split_k(int(on)), "lr_set_split_k")
+    """Split long K loops of small prefill GEMMs over several CTAs (True, the
+    default) or not (False)."""
+    _check(lib().lr_set_split_k(1 if on else 0), "lr_set_split_k")
 
 
 def set_t_precision(mode: int):

@@ -227,10 +227,7 @@ constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
 bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
 
-WaitCtl wait_ctl(DeviceInfo* d) {
-  long long ns = g_wait_ns.load();
-  return WaitCtl{d->status, static_cast<unsigned long long>(ns > 0 ? ns : kDefaultWaitNs)};
-}
+WaitCtl wait_ctl(DeviceInfo* d) { return WaitCtl{d->status, wait_limit_ns()}; }
 
 lr_status validate(const void* X, const void* A, const void* B, const void* bias, const void* Y,
                    int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, bool y_f32 = false) {
@@ -524,53 +521,6 @@ double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
   return *std::max_element(t.begin(), t.end()) + tail;
 }
 
-// The same schedule with the K loop of problem i cut into splits[i] parts
-// (consecutive tiles of the launch).  A split tile's row block is ready once
-// its last part has finished and rounded the partial sums (one more
-// epilogue).
-double simulate_chain_split(const ChainArgs& a, const std::vector<int>& bn,
-                            const std::vector<int>& splits, int sms) {
-  int64_t total = 0;
-  for (int i = 0; i < a.n_prob; ++i)
-    total += ceil_div(a.p[i].Mr, kGemmBM) * ceil_div(a.p[i].Nc, bn[i]) * splits[i];
-  const int64_t G = std::max<int64_t>(1, std::min<int64_t>(total, sms));
-  std::vector<double> t(static_cast<size_t>(G), 0.0);
-  std::map<int, std::vector<double>> ready;
-  int64_t idx = 0;
-  double tail = 0.0;
-  for (int i = 0; i < a.n_prob; ++i) {
-    const ChainProblem& P = a.p[i];
-    const int64_t tm = ceil_div(P.Mr, kGemmBM), tn = ceil_div(P.Nc, bn[i]);
-    const int64_t nkb = ceil_div(P.Kc, kGemmBK);
-    const int64_t per = ceil_div(nkb, splits[i]);
-    const int sp = static_cast<int>(ceil_div(nkb, per));
-    const double fin = sp > 1 ? epilogue_us(bn[i]) : 0.0;
-    std::vector<double>* sig = nullptr;
-    const std::vector<double>* wait = nullptr;
-    if (P.signal_group >= 0) {
-      sig = &ready[P.signal_group];
-      sig->assign(static_cast<size_t>(tm), 0.0);
-    }
-    if (P.wait_group >= 0) {
-      auto it = ready.find(P.wait_group);
-      if (it != ready.end()) wait = &it->second;
-    }
-    for (int64_t l = 0; l < tm * tn; ++l) {
-      const int64_t m = l / tn;
-      for (int k = 0; k < sp; ++k, ++idx) {
-        const int64_t kb = std::min<int64_t>(per, nkb - k * per);
-        double& tc = t[static_cast<size_t>(idx % G)];
-        double start = tc;
-        if (wait && m < static_cast<int64_t>(wait->size())) start = std::max(start, (*wait)[m]);
-        tc = start + static_cast<double>(kb) * kblock_cost(P, bn[i]) + 0.15;
-        if (sig) (*sig)[m] = std::max((*sig)[m], tc + epilogue_us(bn[i]) + fin);
-      }
-    }
-    tail = epilogue_us(bn[i]);
-  }
-  return *std::max_element(t.begin(), t.end()) + tail;
-}
-
 std::mutex g_plan_mu;
 std::map<std::vector<int64_t>, std::vector<int>> g_plans;
 
@@ -647,30 +597,7 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
   }
   // Split K for a GEMM with too few tiles to fill half the SMs and a long
   // K loop (GEMM1 at small ranks): up to one split per 8 k blocks, as many
-  // as fill the SMs.  In mode 2 (lr_set_split_k) a chain's one signalling
-  // GEMM with at least 16 k blocks may also be split 2..4 ways when the
-  // schedule model finishes the launch sooner that way.
-  std::vector<int> model_split(static_cast<size_t>(a.n_prob), 1);
-  if (g_split_k.load() == 2) {
-    int sig = -1, n_sig = 0;
-    for (int i = 0; i < a.n_prob; ++i)
-      if (a.p[i].signal_group >= 0) {
-        sig = i;
-        ++n_sig;
-      }
-    if (n_sig == 1 && ceil_div(a.p[sig].Kc, kGemmBK) >= 16) {
-      double best = simulate_chain_split(a, bn, model_split, d->sms);
-      std::vector<int> trial = model_split;
-      for (int sp = 2; sp <= 4; ++sp) {
-        trial[static_cast<size_t>(sig)] = sp;
-        const double t = simulate_chain_split(a, bn, trial, d->sms);
-        if (t < best * 0.98) {
-          best = t;
-          model_split[static_cast<size_t>(sig)] = sp;
-        }
-      }
-    }
-  }
+  // as fill the SMs.
   int64_t split_floats = 0;
   for (int i = 0; i < a.n_prob; ++i) {
     ChainProblem& P = a.p[i];
@@ -682,8 +609,6 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
     int splits = 1;
     if (g_split_k.load() && tiles * 2 <= d->sms && nkb >= 16)
       splits = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({nkb / 8, d->sms / tiles, 16})));
-    else if (model_split[static_cast<size_t>(i)] > 1)
-      splits = model_split[static_cast<size_t>(i)];
     P.kb_per_split = static_cast<int>(ceil_div(nkb, splits));
     P.splits = static_cast<int>(ceil_div(nkb, P.kb_per_split));
     P.split_group = -1;
@@ -727,7 +652,9 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
   a.pdl = 1;
   a.withhold_first_stage = g_withhold.load();
   const int grid = static_cast<int>(std::min<int64_t>(total, d->sms));
-  return launched(launch_chain(cb.maps, a, grid, stream));
+  bool two = false;
+  for (int i = 0; i < a.n_prob; ++i) two = two || a.p[i].map_a_lo >= 0;
+  return launched(launch_chain(cb.maps, a, grid, two, stream));
 }
 
 // One GEMM on CTA pairs (path 4): C = a · b (+bias).
@@ -914,6 +841,22 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
     note_call(stream, false, Y, ybytes);
     return launched(launch_fill_bias(Y, y_f32, ldy, M, N, static_cast<const __nv_bfloat16*>(bias),
                                      stream));
+  }
+  if (path == 0 && tiny_fits(M, K, r, N)) {
+    note_call(stream, false, Y, ybytes);
+    TinyArgs t{};
+    t.M = static_cast<int>(M);
+    t.K = static_cast<int>(K);
+    t.r = static_cast<int>(r);
+    t.N = static_cast<int>(N);
+    t.X = X;
+    t.A = A;
+    t.B = B;
+    t.bias = static_cast<const __nv_bfloat16*>(bias);
+    t.Y = Y;
+    t.ldy = ldy;
+    t.y_f32 = y_f32 ? 1 : 0;
+    return launched(launch_tiny(t, stream));
   }
   const bool decode = (path == 1) || (path == 0 && M <= 16);
   if (decode) {
@@ -1113,6 +1056,11 @@ bool y_disjoint(const lr_proj& p, const lr_proj& q, int64_t M) {
 }  // namespace
 
 void note_cuda_error(int e) { g_last_cuda_error = e; }
+
+unsigned long long wait_limit_ns() {
+  const long long ns = g_wait_ns.load();
+  return static_cast<unsigned long long>(ns > 0 ? ns : kDefaultWaitNs);
+}
 
 void note_launches(int n) { g_launches += n; }
 
@@ -1344,7 +1292,7 @@ lr_status lr_set_wait_limit_ns(int64_t ns) {
 int64_t lr_kernel_launch_count(void) { return g_launches.load(); }
 
 lr_status lr_set_split_k(int on) {
-  if (on < 0 || on > 2) return LR_ERR_INVALID_ARG;
+  if (on < 0 || on > 1) return LR_ERR_INVALID_ARG;
   g_split_k.store(on);
   return LR_OK;
 }

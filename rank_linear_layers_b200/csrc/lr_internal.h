@@ -25,6 +25,9 @@ cudaError_t static_status_take(unsigned int* code);
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
 cudaError_t ensure_max_smem(const void* kernel, int bytes);
 
+// The time limit of device-side bounded waits (lr_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+
 // ------------------------------------------------------------------ decode
 // out[m, n] = sum_k V[m, k] · W[k, n] for m < M (M <= 16), W a bf16 [Kd, Nd]
 // row-major matrix with row stride ldw.  Split over column blocks (grid.x)
@@ -73,6 +76,25 @@ SkinnyPlan plan_skinny(int M, int64_t Kd, int64_t Nd, int num_sms);
 // first rows of W and then waits for that launch before reading V.
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& args, cudaStream_t stream,
                           bool dependent = false);
+
+// ------------------------------------------------------------------ tiny layers
+// The whole layer in one CTA (lr_tiny.cu) when it fits its shared memory:
+// M <= 16 and small factors.
+struct TinyArgs {
+  int M, K, r, N;
+  const void* X;
+  const void* A;
+  const void* B;
+  const __nv_bfloat16* bias;
+  void* Y;
+  int64_t ldy;
+  int y_f32;
+};
+constexpr size_t kTinyMaxSmem = 200 * 1024;
+__host__ __device__ inline size_t tiny_align16(size_t x) { return (x + 15) / 16 * 16; }
+size_t tiny_smem_bytes(int64_t M, int64_t K, int64_t r, int64_t N);
+bool tiny_fits(int64_t M, int64_t K, int64_t r, int64_t N);
+cudaError_t launch_tiny(const TinyArgs& a, cudaStream_t stream);
 
 // ------------------------------------------------------------------ prefill
 // C[Mr, Nc] = Aop[Mr, Kc] · Bop[Kc, Nc] (+ bias), bf16 in, fp32 accumulate,
@@ -191,7 +213,8 @@ struct ChainMaps {
 };
 
 size_t chain_smem_bytes();
-cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& args, int grid,
+// `two`: some problem of the launch reads operand a in two parts (map_a_lo).
+cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& args, int grid, bool two,
                          cudaStream_t stream);
 
 // Copy a [rows, cols] bf16 matrix with any 2-byte-aligned base and pitch lds

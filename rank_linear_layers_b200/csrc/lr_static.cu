@@ -153,9 +153,13 @@ extern "C" lr_status lr_linear_decode_static(const void* X, const void* A, const
 
   SkinnyArgs a{};
   a.M = m;
-  // Bounded waits report to a status word kept in the same array.
+  // Bounded waits would report to a status word kept in the same array, with
+  // the library's wait limit (lr_set_wait_limit_ns).  The decode kernels have
+  // none today (their one wait, for the previous launch's grid, is resolved
+  // by the hardware), so the word stays zero; lr_last_device_status reads it
+  // all the same.
   a.wait = WaitCtl{reinterpret_cast<DevStatus*>(scratch + kStaticBytes - kStatusBytes),
-                   2000000000ull};
+                   wait_limit_ns()};
   // Phase 1: T = X·A (fp32).
   a.Kd = K;
   a.Nd = r;

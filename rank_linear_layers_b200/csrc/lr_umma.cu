@@ -275,6 +275,9 @@ __device__ bool wait_rows_ready(const ChainArgs& g, int grp, int m_blk, int coun
   return true;
 }
 
+// kTwo: some problem reads operand a in two parts; without it the two-part
+// code is compiled out of the copy and MMA loops.
+template <bool kTwo>
 __global__ void __launch_bounds__(kChainThreads, 1)
     umma_chain_kernel(const __grid_constant__ ChainMaps maps, const __grid_constant__ ChainArgs g) {
   extern __shared__ uint8_t smem_raw[];
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         const int m_blk = otile / P.tiles_n, n_blk = otile - m_blk * P.tiles_n;
         const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
         const int nbox = (P.bn + 63) / 64;
-        const bool two = P.map_a_lo >= 0;  // bn <= 128: the low part goes after the b tile
+        const bool two = kTwo && P.map_a_lo >= 0;  // bn <= 128: the low part goes after the b tile
         const uint32_t bytes = (two ? 2 : 1) * A_STAGE + nbox * B_ATOM;
         const CUtensorMap* ma = &maps.m[P.map_a];
         const CUtensorMap* ma_lo = two ? &maps.m[P.map_a_lo] : nullptr;
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       const int kbase = (local - (local / P.splits) * P.splits) * P.kb_per_split;
       const int num_kb = min((P.Kc + BK - 1) / BK - kbase, P.kb_per_split);
       const uint32_t idesc = idesc_bf16_f32(BM, P.bn, false, true);
-      const bool two = P.map_a_lo >= 0;
+      const bool two = kTwo && P.map_a_lo >= 0;
       const int acc = it & 1;
       const uint32_t aph = static_cast<uint32_t>(it >> 1) & 1u;
       if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait, kWhereMmaAcc)) {
@@ -836,11 +839,12 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, const GemmMaps& maps, int num_sm
   return cudaGetLastError();
 }
 
-cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid,
+cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid, bool two,
                          cudaStream_t stream) {
   const size_t smem = chain_smem_bytes();
-  cudaError_t e =
-      ensure_max_smem(reinterpret_cast<const void*>(umma_chain_kernel), static_cast<int>(smem));
+  const void* kern = two ? reinterpret_cast<const void*>(umma_chain_kernel<true>)
+                         : reinterpret_cast<const void*>(umma_chain_kernel<false>);
+  cudaError_t e = ensure_max_smem(kern, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(std::max(1, grid));
@@ -852,7 +856,8 @@ cudaError_t launch_chain(const ChainMaps& maps, const ChainArgs& g, int grid,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = g.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, umma_chain_kernel, maps, g);
+  if (two) return cudaLaunchKernelEx(&cfg, umma_chain_kernel<true>, maps, g);
+  return cudaLaunchKernelEx(&cfg, umma_chain_kernel<false>, maps, g);
 }
 
 cudaError_t launch_fill_bias(void* Y, bool y_f32, int64_t ldy, int64_t M, int64_t N,

@@ -95,10 +95,13 @@ def test_controls(L):
         assert L.lr_set_tile_n(bad) == lr.LR_ERR_INVALID_ARG
     for ok in (32, 96, 256, 0):
         assert L.lr_set_tile_n(ok) == lr.LR_OK
-    for bad in (-1, 3):
+    for bad in (-1, 2, 3):
         assert L.lr_set_split_k(bad) == lr.LR_ERR_INVALID_ARG
-    assert L.lr_set_split_k(2) == lr.LR_OK
     assert L.lr_set_split_k(0) == lr.LR_OK and L.lr_set_split_k(1) == lr.LR_OK
+    for bad in (-1, 3):
+        assert L.lr_set_t_precision(bad) == lr.LR_ERR_INVALID_ARG
+    for ok in (1, 2, 0):
+        assert L.lr_set_t_precision(ok) == lr.LR_OK
     for bad in (-1, 2):
         assert L.lr_set_early_copy(bad) == lr.LR_ERR_INVALID_ARG
     assert L.lr_set_early_copy(0) == lr.LR_OK and L.lr_set_early_copy(1) == lr.LR_OK

@@ -40,8 +40,14 @@ def test_decoder_layer_group(M, n_int):
         else:
             e["Y"] = Ys[n]
         entries.append(e)
-    lr.lr_linear_group(entries, M)
-    torch.cuda.synchronize()
+    # Tiles whole (no K range split between SMs), so that the group and the
+    # single calls form every sum in the same order.
+    lr.set_split_k(False)
+    try:
+        lr.lr_linear_group(entries, M)
+        torch.cuda.synchronize()
+    finally:
+        lr.set_split_k(True)
     assert lr.last_device_status() == lr.LR_OK
     outs = {n: to_f64(Ys[n]) for n in Ys}
     pk = to_f64(packed)
@@ -49,14 +55,11 @@ def test_decoder_layer_group(M, n_int):
     for n, p in P.items():
         X = layer["inputs"][p["x"]]
         # The same projection through lr_linear alone: the same bits on the
-        # prefill path; on the decode path fp32 atomics may add partial sums
-        # in another order, so compare at the parity tolerance there.
+        # prefill path (tiles whole in both: tiling differs, sums do not); on
+        # the decode path fp32 atomics may add partial sums in another order,
+        # so compare at the parity tolerance there.
         A, B = dev[n]
         if M > 16:
-            # Without split K the single call does the same arithmetic per
-            # output element (tiling differs, sums do not); with split K
-            # (the default) fp32 reductions may add partial sums in another
-            # order.
             lr.set_split_k(False)
             try:
                 Y1 = to_f64(lr.lr_linear(xs[p["x"]], A, B))
@@ -72,7 +75,7 @@ def test_decoder_layer_group(M, n_int):
             compare(outs[n], Y1, f"group vs single {n}")
 
 
-def _group_case(specs, M, seed):
+def _group_case(specs, M, seed, split=True):
     """specs: list of (x_name, K, r, N, bias).  Returns inputs, entries, outputs."""
     import torch
     import rank_linear_layers_b200 as lr
@@ -89,8 +92,12 @@ def _group_case(specs, M, seed):
         entries.append(e)
         outs.append(Y)
         probs.append(p)
-    lr.lr_linear_group(entries, M)
-    torch.cuda.synchronize()
+    lr.set_split_k(split)
+    try:
+        lr.lr_linear_group(entries, M)
+        torch.cuda.synchronize()
+    finally:
+        lr.set_split_k(True)
     assert lr.last_device_status() == lr.LR_OK
     return entries, outs, probs
 
@@ -99,7 +106,8 @@ def _group_case(specs, M, seed):
 def test_group_sets_share_x(M):
     """Sets of projections sharing X (concatenated factors, one GEMM1 per set,
     one launch), odd ranks and K, a misaligned X, bias on some: every output
-    equals the oracle, and bit for bit the projection run alone."""
+    equals the oracle (tiles split along K between SMs, the default) and,
+    with every tile whole, bit for bit the projection run alone."""
     import rank_linear_layers_b200 as lr
     specs = [("x1", 136, 37, 100, False), ("x1", 136, 64, 64, False), ("x1", 136, 5, 517, True),
              ("x2", 333, 257, 40, True), ("x2", 333, 1, 8, False), ("x3", 64, 7, 9, False),
@@ -108,8 +116,14 @@ def test_group_sets_share_x(M):
     for e, Y, p in zip(entries, outs, probs):
         compare(to_f64(Y), oracle.lr_linear(p["X"], p["A"], p["B"], p.get("bias")),
                 f"group K={p['K']} r={p['r']} N={p['N']}")
-        Y1 = lr.lr_linear(e["X"], e["A"], e["B"], e.get("bias"))
-        assert np.array_equal(to_f64(Y1), to_f64(Y)), f"group vs single r={p['r']}"
+    entries, outs, probs = _group_case(specs, M, seed=40, split=False)
+    lr.set_split_k(False)
+    try:
+        for e, Y, p in zip(entries, outs, probs):
+            Y1 = lr.lr_linear(e["X"], e["A"], e["B"], e.get("bias"))
+            assert np.array_equal(to_f64(Y1), to_f64(Y)), f"group vs single r={p['r']}"
+    finally:
+        lr.set_split_k(True)
 
 
 def test_group_larger_than_one_launch():

@@ -69,6 +69,28 @@ def test_decode_shapes(lr, K, N):
     compare(run_gpu(lr, p, lr.PATH_DECODE), ref(p), f"decode16 K={K} N={N}")
 
 
+@pytest.mark.parametrize("M,K,r,N", [(1, 333, 57, 77), (5, 256, 107, 256), (16, 200, 33, 517),
+                                     (16, 1000, 9, 130), (3, 64, 1, 8)])
+def test_tiny_layer_one_cta(lr, M, K, r, N):
+    """Small layers (automatic dispatch): the whole layer in one CTA, odd
+    sizes and bias, bf16 and fp32 outputs, operands not 16-byte aligned."""
+    import torch
+    p = lrgen.lowrank_problem(M, K, r, N, seed=M * 7 + r, bias=True)
+    Yr = ref(p)
+    n0 = lr.kernel_launch_count()
+    compare(run_gpu(lr, p), Yr, f"tiny {M}x{K}x{r}x{N}")
+    assert lr.kernel_launch_count() - n0 == 1
+
+    def off(bits):
+        t = to_dev(bits).reshape(-1)
+        buf = torch.empty(t.numel() + 1, dtype=torch.bfloat16, device="cuda")
+        buf[1:] = t
+        return buf[1:].view(bits.shape)
+    Y32 = lr.lr_linear_f32(off(p["X"]), off(p["A"]), off(p["B"]), off(p["bias"]))
+    torch.cuda.synchronize()
+    compare(f32_host(Y32), Yr, "tiny fp32, unaligned operands")
+
+
 # ---------------------------------------------------------------- prefill
 @pytest.mark.parametrize("M,K,r,N", [
     (128, 64, 64, 256),       # one tile each way, all aligned

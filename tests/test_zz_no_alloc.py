@@ -3,10 +3,11 @@ library allocate device memory (a serving loop that cannot afford the device
 synchronisation cudaMalloc/cudaFree cause, or a host whose own pool owns all
 device memory).  Its scratch is a fixed array inside the library.
 
-Checked through the C ABI against lr_linear (the allocating entry point) on
-the same inputs, at the parity tolerance used everywhere else, on two calls
-in a row (the array keeps the previous call's contents, so the second call
-also checks that it is cleared).  This file is collected last on purpose.
+Checked through the C ABI, on two calls in a row (the array keeps the
+previous call's contents), against the fp64 oracle and against lr_linear
+(the allocating entry point) on the same inputs, at the parity tolerance
+used everywhere else; the device's free memory is the same before and after
+the calls.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 
 import lrgen
+import oracle
 from helpers import compare, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -46,11 +48,22 @@ def test_static_matches_allocating_entry_point(M, K, r, N, with_bias):
                        None if b is None else b.data_ptr(), Yref.data_ptr(), M, K, r, N,
                        stream) == lr.LR_OK
     ref = to_f64(Yref)
+    Yo = oracle.lr_linear(p["X"], p["A"], p["B"], p["bias"])
+    Ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    # The first call on a device looks up the array's address; after it the
+    # calls allocate nothing: free device memory is unchanged.
+    assert _call_static(L, X, A, B, b, Ys[0], M, K, r, N, stream) == lr.LR_OK
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     for call in range(2):
-        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        Y = Ys[call]
+        Y.fill_(float("nan"))
         assert _call_static(L, X, A, B, b, Y, M, K, r, N, stream) == lr.LR_OK
         torch.cuda.synchronize()
-        compare(to_f64(Y), ref, f"static call {call} M={M} K={K} r={r} N={N}")
+        compare(to_f64(Y), Yo, f"static call {call} vs oracle M={M} K={K} r={r} N={N}")
+        compare(to_f64(Y), ref, f"static call {call} vs lr_linear M={M} K={K} r={r} N={N}")
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert lr.last_device_status() == lr.LR_OK
 
 
 def test_static_rejects_sizes_beyond_its_array():
