@@ -113,6 +113,32 @@ lr_status lr_linear_f32(const void* X, const void* A, const void* B, const void*
                         int64_t M, int64_t K, int64_t r, int64_t N, void* stream);
 
 /*
+ * lr_linear_strided — lr_linear on row-major operands with any row pitches
+ * (elements): X [M,K] pitch ldx >= K, A [K,r] pitch lda >= r, B [r,N] pitch
+ * ldb >= N, Y [M,N] pitch ldy >= N; Y is bf16 (y_f32 = 0) or fp32
+ * (y_f32 != 0, as lr_linear_f32).  Same paths and results as lr_linear.
+ *
+ * A prefill operand whose base is 32-byte aligned and whose pitch is a
+ * multiple of 16 elements is read in place; any other is first copied to an
+ * aligned pitch on every call (for a factor with r = 1741, 14 MB per call).
+ * A caller that keeps its factors in buffers of pitch lr_factor_pitch(cols)
+ * (cudaMalloc bases are 256-byte aligned) pays that copy once, when it
+ * stores them, instead of on every call: the "prepared weight" form of a
+ * static factor.  Not this library's allocation: the caller owns those
+ * buffers.
+ */
+lr_status lr_linear_strided(const void* X, int64_t ldx, const void* A, int64_t lda, const void* B,
+                            int64_t ldb, const void* bias, void* Y, int64_t ldy, int64_t M,
+                            int64_t K, int64_t r, int64_t N, int32_t y_f32, void* stream);
+
+/*
+ * lr_factor_pitch — the row pitch (elements) at which a stored factor with
+ * `cols` columns is read in place by the prefill path: cols rounded up to a
+ * multiple of 64 (128-byte rows).  -1 for cols < 0.
+ */
+int64_t lr_factor_pitch(int64_t cols);
+
+/*
  * One projection of a group (a decoder layer's q/k/v/o/gate/up/down).
  * X [M,K] (entries may share one X pointer), A [K,r], B [r,N], bias [N] or
  * NULL, Y with row stride ld_y >= N (so two projections can write the two

@@ -35,7 +35,7 @@ EXPORTS = (
     "lr_status_string", "lr_last_cuda_error", "lr_set_path", "lr_set_wait_limit_ns",
     "lr_kernel_launch_count", "lr_release_workspaces", "lr_linear_decode_static",
     "lr_set_withhold_first_stage", "lr_set_tile_n", "lr_set_split_k", "lr_set_early_copy",
-    "lr_gac_select", "lr_set_t_precision",
+    "lr_gac_select", "lr_set_t_precision", "lr_linear_strided", "lr_factor_pitch",
 )
 
 T_AUTO, T_BF16, T_TWO_PARTS = 0, 1, 2
@@ -73,6 +73,10 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, i64 = ctypes.c_void_p, ctypes.c_int64
     L.lr_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_linear_f32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    L.lr_linear_strided.argtypes = [vp, i64, vp, i64, vp, i64, vp, vp, i64, i64, i64, i64, i64,
+                                    ctypes.c_int32, vp]
+    L.lr_factor_pitch.argtypes = [i64]
+    L.lr_factor_pitch.restype = i64
     L.lr_linear_group.argtypes = [ctypes.POINTER(LrProj), ctypes.c_int, i64, vp]
     L.lr_linear_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     L.lr_dense.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
@@ -94,7 +98,8 @@ def lib(path: str = LIB_PATH) -> ctypes.CDLL:
     L.lr_kernel_launch_count.argtypes = []
     L.lr_kernel_launch_count.restype = i64
     L.lr_release_workspaces.argtypes = []
-    for name in ("lr_linear", "lr_linear_f32", "lr_linear_group", "lr_linear_host", "lr_dense",
+    for name in ("lr_linear", "lr_linear_f32", "lr_linear_strided", "lr_linear_group",
+                 "lr_linear_host", "lr_dense",
                  "lr_linear_decode_static",
                  "lr_last_device_status", "lr_last_cuda_error", "lr_set_path",
                  "lr_set_wait_limit_ns", "lr_release_workspaces", "lr_set_withhold_first_stage",
@@ -178,6 +183,37 @@ def lr_linear_f32(X, A, B, bias=None, Y=None, stream=None):
     _check(lib().lr_linear_f32(_ptr(X), _ptr(A), _ptr(B), _ptr(bias), _ptr(Y), M, K, r, N,
                                _stream_ptr(stream)), "lr_linear_f32")
     return Y
+
+
+def lr_linear_strided(X, A, B, bias=None, Y=None, stream=None):
+    """lr_linear on 2-D views with row strides (element stride 1): for
+    instance a factor stored in a buffer of pitch lr_factor_pitch(r) and
+    passed as buf[:, :r].  Y bf16 or fp32 (allocated bf16 if None)."""
+    import torch
+    M, K = X.shape
+    r = A.shape[1]
+    N = B.shape[1]
+    for name, t in (("X", X), ("A", A), ("B", B)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(1) != 1:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor with unit column stride")
+    if A.shape[0] != K or B.shape[0] != r:
+        raise ValueError("shapes do not chain")
+    _check_bf16("bias", bias, (N,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if Y.dtype not in (torch.bfloat16, torch.float32) or not Y.is_cuda or Y.stride(1) != 1 or \
+            tuple(Y.shape) != (M, N):
+        raise TypeError("Y must be a bf16 or fp32 CUDA tensor (M, N) with unit column stride")
+    _check(lib().lr_linear_strided(_ptr(X), X.stride(0), _ptr(A), A.stride(0), _ptr(B),
+                                   B.stride(0), _ptr(bias), _ptr(Y), Y.stride(0), M, K, r, N,
+                                   1 if Y.dtype == torch.float32 else 0, _stream_ptr(stream)),
+           "lr_linear_strided")
+    return Y
+
+
+def factor_pitch(cols: int) -> int:
+    """Row pitch (elements) at which a stored factor is read in place."""
+    return int(lib().lr_factor_pitch(int(cols)))
 
 
 def lr_dense(X, W, bias=None, Y=None, stream=None):

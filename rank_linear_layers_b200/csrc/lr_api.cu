@@ -229,20 +229,28 @@ bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0
 
 WaitCtl wait_ctl(DeviceInfo* d) { return WaitCtl{d->status, wait_limit_ns()}; }
 
+// Row pitches (elements) of X, A and B; contiguous unless a caller says so.
+struct Pitch {
+  int64_t x, a, b;
+};
+
 lr_status validate(const void* X, const void* A, const void* B, const void* bias, const void* Y,
-                   int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, bool y_f32 = false) {
+                   int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, bool y_f32 = false,
+                   Pitch ld = Pitch{-1, -1, -1}) {
   if (M < 0 || K < 0 || r < 0 || N < 0) return LR_ERR_INVALID_ARG;
   if (M > kMaxDim || K > kMaxDim || r > kMaxDim || N > kMaxDim) return LR_ERR_UNSUPPORTED;
-  if (ldy < N) return LR_ERR_INVALID_ARG;
+  if (ld.x < 0) ld = Pitch{K, r, N};
+  if (ldy < N || ld.x < K || ld.a < r || ld.b < N) return LR_ERR_INVALID_ARG;
+  if (ldy > kMaxDim || ld.x > kMaxDim || ld.a > kMaxDim || ld.b > kMaxDim) return LR_ERR_UNSUPPORTED;
   if (M > 0 && N > 0 && !Y) return LR_ERR_INVALID_ARG;
   if (M > 0 && K > 0 && r > 0 && N > 0 && (!X || !A || !B)) return LR_ERR_INVALID_ARG;
   for (const void* p : {X, A, B, bias, Y})
     if (p && !aligned2(p)) return LR_ERR_INVALID_ARG;
   if (y_f32 && Y && (reinterpret_cast<uintptr_t>(Y) & 3u) != 0) return LR_ERR_INVALID_ARG;
   const size_t ybytes = span_bytes(M, N, ldy) * (y_f32 ? 2 : 1);
-  if (ranges_overlap(Y, ybytes, X, span_bytes(M, K, K)) ||
-      ranges_overlap(Y, ybytes, A, span_bytes(K, r, r)) ||
-      ranges_overlap(Y, ybytes, B, span_bytes(r, N, N)) ||
+  if (ranges_overlap(Y, ybytes, X, span_bytes(M, K, ld.x)) ||
+      ranges_overlap(Y, ybytes, A, span_bytes(K, r, ld.a)) ||
+      ranges_overlap(Y, ybytes, B, span_bytes(r, N, ld.b)) ||
       ranges_overlap(Y, ybytes, bias, span_bytes(1, N, N)))
     return LR_ERR_INVALID_ARG;
   return LR_OK;
@@ -258,7 +266,8 @@ lr_status launched(cudaError_t e, int n = 1) {
 lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64_t ldv, bool v_f32,
                  const void* W, int64_t Kd, int64_t Nd, float* acc, unsigned int* counters,
                  float* out_f32, int64_t ld_out_f32, void* out_bf16, int64_t ld_out,
-                 const void* bias, bool dependent = false) {
+                 const void* bias, bool dependent = false, int64_t ldw = -1) {
+  if (ldw < 0) ldw = Nd;
   const SkinnyPlan plan = plan_skinny(M, Kd, Nd, d->sms);
   SkinnyArgs a{};
   a.M = M;
@@ -268,9 +277,9 @@ lr_status skinny(DeviceInfo* d, cudaStream_t stream, int M, const void* V, int64
   a.ldv = ldv;
   a.v_f32 = v_f32 ? 1 : 0;
   a.W = static_cast<const __nv_bfloat16*>(W);
-  a.ldw = Nd;
+  a.ldw = ldw;
   a.w_lo = reinterpret_cast<uintptr_t>(W);
-  a.w_hi = a.w_lo + static_cast<uintptr_t>(Kd * Nd * 2);
+  a.w_hi = a.w_lo + static_cast<uintptr_t>(span_bytes(Kd, Nd, ldw));
   a.acc = acc;
   a.ld_acc = static_cast<int64_t>(align_up(static_cast<size_t>(Nd), 4));
   a.counters = counters;
@@ -291,7 +300,7 @@ size_t ctr_bytes(int M, int64_t Kd, int64_t n, int sms) {
 
 lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                      const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
-                     int64_t N, int64_t ldy, bool y_f32) {
+                     int64_t N, int64_t ldy, bool y_f32, Pitch ld) {
   const int m = static_cast<int>(M);
   const size_t acc1 = acc_bytes(m, r), acc2 = acc_bytes(m, N);
   const size_t c1 = ctr_bytes(m, K, r, d->sms), c2 = ctr_bytes(m, r, N, d->sms);
@@ -306,14 +315,15 @@ lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const vo
   unsigned int* k2 = reinterpret_cast<unsigned int*>(zero + acc1 + acc2 + c1);
   float* T = reinterpret_cast<float*>(scratch);
   // Phase 1: T = X·A (fp32).  Phase 2: Y = T·B + bias.
-  st = skinny(d, stream, m, X, K, false, A, K, r, a1, k1, T, ldt, nullptr, 0, nullptr);
+  st = skinny(d, stream, m, X, ld.x, false, A, K, r, a1, k1, T, ldt, nullptr, 0, nullptr, false,
+              ld.a);
   if (st != LR_OK) return st;
   // Phase 2 starts streaming B while phase 1 finishes (programmatic
   // dependent launch); it reads T only after phase 1 has completed.
   if (y_f32)
     return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, static_cast<float*>(Y), ldy,
-                  nullptr, 0, bias, true);
-  return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias, true);
+                  nullptr, 0, bias, true, ld.b);
+  return skinny(d, stream, m, T, ldt, true, B, r, N, a2, k2, nullptr, 0, Y, ldy, bias, true, ld.b);
 }
 
 // Row pitch (elements) of the buffers the library lays out itself (T and
@@ -741,10 +751,11 @@ bool t_in_two_parts(int64_t M, int64_t K, int64_t r, int64_t N) {
 
 lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                       const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
-                      int64_t N, int64_t ldy, bool y_f32) {
+                      int64_t N, int64_t ldy, bool y_f32, Pitch ld) {
   const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), kPitchElems));
   const size_t tbytes = align_up(static_cast<size_t>(M) * ldt * 2, 256);
-  const size_t rp = repack_bytes(X, K, M, K) + repack_bytes(A, r, K, r) + repack_bytes(B, N, r, N);
+  const size_t rp = repack_bytes(X, ld.x, M, K) + repack_bytes(A, ld.a, K, r) +
+                    repack_bytes(B, ld.b, r, N);
   const bool pairs = g_path.load() == 4;
   if (pairs && y_f32) return LR_ERR_UNSUPPORTED;
   const bool two = !pairs && t_in_two_parts(M, K, r, N);
@@ -763,15 +774,16 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
   bool early = false;
   if (rp > 0 && !pairs) {
     st = repack_area(stream, rp,
-                     {{X, span_bytes(M, K, K)}, {A, span_bytes(K, r, r)}, {B, span_bytes(r, N, N)}},
+                     {{X, span_bytes(M, K, ld.x)}, {A, span_bytes(K, r, ld.a)},
+                      {B, span_bytes(r, N, ld.b)}},
                      &scratch, &early);
     if (st != LR_OK) return st;
   }
   Operand x, a, b;
   int repacks = 0;
-  if ((st = tma_operand(d, stream, X, K, M, K, &scratch, &x, &repacks, early)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, A, r, K, r, &scratch, &a, &repacks, early)) != LR_OK) return st;
-  if ((st = tma_operand(d, stream, B, N, r, N, &scratch, &b, &repacks, early)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, X, ld.x, M, K, &scratch, &x, &repacks, early)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, A, ld.a, K, r, &scratch, &a, &repacks, early)) != LR_OK) return st;
+  if ((st = tma_operand(d, stream, B, ld.b, r, N, &scratch, &b, &repacks, early)) != LR_OK) return st;
   if (pairs) {
     // CTA-pair tiles: the two GEMMs as two launches.
     note_call(stream, false, Y, span_bytes(M, N, ldy));
@@ -826,8 +838,9 @@ lr_status run_prefill(DeviceInfo* d, cudaStream_t stream, const void* X, const v
 
 lr_status run_linear(const void* X, const void* A, const void* B, const void* bias, void* Y,
                      int64_t M, int64_t K, int64_t r, int64_t N, int64_t ldy, cudaStream_t stream,
-                     bool y_f32 = false) {
-  lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
+                     bool y_f32 = false, Pitch ld = Pitch{-1, -1, -1}) {
+  if (ld.x < 0) ld = Pitch{K, r, N};
+  lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy, y_f32, ld);
   if (st != LR_OK) return st;
   const int path = g_path.load();
   if (path == 1 && M > 16) return LR_ERR_INVALID_ARG;
@@ -842,7 +855,8 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
     return launched(launch_fill_bias(Y, y_f32, ldy, M, N, static_cast<const __nv_bfloat16*>(bias),
                                      stream));
   }
-  if (path == 0 && tiny_fits(M, K, r, N)) {
+  const bool contiguous = ld.x == K && ld.a == r && ld.b == N;
+  if (path == 0 && contiguous && tiny_fits(M, K, r, N)) {
     note_call(stream, false, Y, ybytes);
     TinyArgs t{};
     t.M = static_cast<int>(M);
@@ -861,9 +875,9 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
   const bool decode = (path == 1) || (path == 0 && M <= 16);
   if (decode) {
     note_call(stream, false, Y, ybytes);
-    return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
+    return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32, ld);
   }
-  return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32);
+  return run_prefill(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32, ld);
 }
 
 
@@ -1095,6 +1109,18 @@ lr_status lr_linear(const void* X, const void* A, const void* B, const void* bia
 lr_status lr_linear_f32(const void* X, const void* A, const void* B, const void* bias, void* Y,
                         int64_t M, int64_t K, int64_t r, int64_t N, void* stream) {
   return run_linear(X, A, B, bias, Y, M, K, r, N, N, static_cast<cudaStream_t>(stream), true);
+}
+
+lr_status lr_linear_strided(const void* X, int64_t ldx, const void* A, int64_t lda, const void* B,
+                            int64_t ldb, const void* bias, void* Y, int64_t ldy, int64_t M,
+                            int64_t K, int64_t r, int64_t N, int32_t y_f32, void* stream) {
+  return run_linear(X, A, B, bias, Y, M, K, r, N, ldy, static_cast<cudaStream_t>(stream),
+                    y_f32 != 0, Pitch{ldx, lda, ldb});
+}
+
+int64_t lr_factor_pitch(int64_t cols) {
+  if (cols < 0) return -1;
+  return (cols + kPitchElems - 1) / kPitchElems * kPitchElems;
 }
 
 lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream) {

@@ -10,11 +10,11 @@
 // with asynchronous 16-byte copies (the aligned 16-byte chunks that cover
 // each tensor, so any base alignment and any row pitch work), computes
 // T = X·A in fp32 (kept in shared memory, never rounded), then Y = T·B +
-// bias, and stores Y.  A thread takes one output column for all 16 token
-// rows (X and T are held transposed, so one 16-byte load feeds four FMAs)
-// over one of up to four contiguous k ranges; the ranges' partial sums are
-// added in order.  Every product is an fp32 FMA (packed two rows at a time)
-// of the exact inputs.
+// bias, and stores Y.  Both products run on mma.sync m16n8k16 (the 16 token
+// rows are the MMA's M; bf16 in, fp32 accumulate), each warp taking
+// (8-column tile, k range) tasks whose partial sums are added in k-range
+// order.  T enters the second product as two bf16 parts, hi = bf16(T) and
+// lo = bf16(T - hi), so it keeps about 16 bits, as the decode path does.
 #include <algorithm>
 
 #include "lr_internal.h"
@@ -44,75 +44,109 @@ __device__ __forceinline__ uint32_t stage_raw(uint8_t* dst, const void* p, size_
   return static_cast<uint32_t>(reinterpret_cast<uintptr_t>(p) - lo);
 }
 
-__device__ __forceinline__ float bf(const uint8_t* base, uint32_t off, int64_t idx) {
-  return __bfloat162float(
-      *reinterpret_cast<const __nv_bfloat16*>(base + off + static_cast<uint32_t>(idx) * 2u));
+__device__ __forceinline__ uint32_t bf_bits(const uint8_t* base, uint32_t off, int64_t idx) {
+  return *reinterpret_cast<const unsigned short*>(base + off + static_cast<uint32_t>(idx) * 2u);
 }
 
-// Splits of the reduction dimension so that the threads have work: a thread
-// takes one output column and one of `split` contiguous k ranges.
-__host__ __device__ inline int tiny_split(int cols) {
-  const int s = kTinyThreads / (cols > 0 ? cols : 1);
-  return s < 1 ? 1 : (s > 4 ? 4 : s);
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Shared memory layout (16-byte aligned parts): Xt [K][16] fp32 (X transposed,
-// rows past M zero), Tt [r][16] fp32 (T transposed), partial sums
-// [split][16][cols] fp32, then the raw 16-byte chunks covering A and B.
+// Splits of a product's k steps over warps, so that every warp has work.
+__host__ __device__ inline int tiny_ksplit(int n_tiles, int k_steps) {
+  int s = (16 + n_tiles - 1) / n_tiles;
+  if (s > k_steps) s = k_steps;
+  if (s > 4) s = 4;
+  return s < 1 ? 1 : s;
+}
+
+// Shared memory layout (16-byte aligned parts): X as bf16 [16][kp] (kp = K
+// rounded up to 16, zero past K and M), T's bf16 hi and lo parts [16][rp]
+// (rp = r rounded up to 16, zero past r), T fp32 [16][r], partial sums
+// [splits][16][cols], then the raw 16-byte chunks covering A and B.
 struct TinyLayout {
-  size_t xt, tt, part, araw, braw, total;
+  size_t xs, th, tl, t, part, araw, braw, total;
+  int kp, rp;
 };
 
 __host__ __device__ inline TinyLayout tiny_layout(int64_t K, int64_t r, int64_t N) {
   TinyLayout L;
-  L.xt = 0;
-  L.tt = L.xt + tiny_align16(static_cast<size_t>(K) * 16 * 4);
-  L.part = L.tt + tiny_align16(static_cast<size_t>(r) * 16 * 4);
-  const size_t pt = static_cast<size_t>(tiny_split(static_cast<int>(r))) * 16 * r * 4;
-  const size_t py = static_cast<size_t>(tiny_split(static_cast<int>(N))) * 16 * N * 4;
-  L.araw = L.part + tiny_align16(pt > py ? pt : py);
+  L.kp = static_cast<int>((K + 15) / 16 * 16);
+  L.rp = static_cast<int>((r + 15) / 16 * 16);
+  L.xs = 0;
+  L.th = L.xs + tiny_align16(static_cast<size_t>(16) * L.kp * 2);
+  L.tl = L.th + tiny_align16(static_cast<size_t>(16) * L.rp * 2);
+  L.t = L.tl + tiny_align16(static_cast<size_t>(16) * L.rp * 2);
+  L.part = L.t + tiny_align16(static_cast<size_t>(16) * r * 4);
+  const int nt1 = static_cast<int>((r + 7) / 8), nt2 = static_cast<int>((N + 7) / 8);
+  const size_t p1 = static_cast<size_t>(tiny_ksplit(nt1, L.kp / 16)) * 16 * nt1 * 8 * 4;
+  const size_t p2 = static_cast<size_t>(tiny_ksplit(nt2, L.rp / 16)) * 16 * nt2 * 8 * 4;
+  L.araw = L.part + tiny_align16(p1 > p2 ? p1 : p2);
   L.braw = L.araw + tiny_align16(static_cast<size_t>(K) * r * 2 + 32);
   L.total = L.braw + tiny_align16(static_cast<size_t>(r) * N * 2 + 32);
   return L;
 }
 
-// out[m][c] for m < 16, c < cols: sum over k < depth of vt[k][m] · W[k][c]
-// (W raw bf16 at wbase + woff, row pitch ldw), k split in `split` ranges whose
-// partial sums are added in range order; result to outt[c][m] (transposed)
-// or handed to `store`.
+// out[16][cols] = V[16][depth] · W[depth][cols] on mma.m16n8k16: V from
+// bf16 rows (vh, and vl as a second part when non-null) of pitch vp
+// (zero-padded to a multiple of 16), W from raw bf16 (wbase + woff, row
+// pitch ldw; entries past depth or cols read as zero).  Warps take
+// (n tile, k range) tasks; the k ranges' partial sums are added in order and
+// handed to store(m, c, value).
 template <typename Store>
-__device__ __forceinline__ void tiny_product(const float* vt, const uint8_t* wbase, uint32_t woff,
-                                             int64_t ldw, int depth, int cols, float* part,
-                                             Store store) {
-  const int split = tiny_split(cols);
-  for (int task = threadIdx.x; task < cols * split; task += kTinyThreads) {
-    const int c = task % cols, sp = task / cols;
-    const int k0 = depth * sp / split, k1 = depth * (sp + 1) / split;
-    float2 acc[8];  // rows (2i, 2i + 1), packed fp32x2 FMA
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
-    for (int k = k0; k < k1; ++k) {
-      const float w = bf(wbase, woff, static_cast<int64_t>(k) * ldw + c);
-      const float2 w2 = make_float2(w, w);
-      const float4* v = reinterpret_cast<const float4*>(vt + k * 16);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 x = v[q];
-        acc[2 * q] = __ffma2_rn(make_float2(x.x, x.y), w2, acc[2 * q]);
-        acc[2 * q + 1] = __ffma2_rn(make_float2(x.z, x.w), w2, acc[2 * q + 1]);
+__device__ __forceinline__ void tiny_mma_product(const uint16_t* vh, const uint16_t* vl, int vp,
+                                                 const uint8_t* wbase, uint32_t woff, int64_t ldw,
+                                                 int depth, int cols, float* part, Store store) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int nt = (cols + 7) / 8, ks = (depth + 15) / 16;
+  const int split = tiny_ksplit(nt, ks);
+  for (int task = warp; task < nt * split; task += kTinyThreads / 32) {
+    const int n_tile = task % nt, sp = task / nt;
+    const int k0 = ks * sp / split, k1 = ks * (sp + 1) / split;
+    const int n = n_tile * 8 + g;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int kstep = k0; kstep < k1; ++kstep) {
+      const int kb = kstep * 16;
+      auto afrag = [&](const uint16_t* v, uint32_t (&a)[4]) {
+        const uint32_t* r0 = reinterpret_cast<const uint32_t*>(v + g * vp + kb);
+        const uint32_t* r8 = reinterpret_cast<const uint32_t*>(v + (g + 8) * vp + kb);
+        a[0] = r0[t];
+        a[1] = r8[t];
+        a[2] = r0[t + 4];
+        a[3] = r8[t + 4];
+      };
+      auto w = [&](int k) -> uint32_t {
+        return (k < depth && n < cols) ? bf_bits(wbase, woff, static_cast<int64_t>(k) * ldw + n) : 0u;
+      };
+      const uint32_t b0 = w(kb + 2 * t) | (w(kb + 2 * t + 1) << 16);
+      const uint32_t b1 = w(kb + 2 * t + 8) | (w(kb + 2 * t + 9) << 16);
+      uint32_t a[4];
+      afrag(vh, a);
+      mma16816(d, a, b0, b1);
+      if (vl) {
+        afrag(vl, a);
+        mma16816(d, a, b0, b1);
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      part[(sp * 16 + 2 * i) * cols + c] = acc[i].x;
-      part[(sp * 16 + 2 * i + 1) * cols + c] = acc[i].y;
-    }
+    // C fragment: rows g, g + 8; columns 2t, 2t + 1 of the n tile.
+    float* pp = part + static_cast<int64_t>(sp) * 16 * nt * 8;
+    const int c = n_tile * 8 + 2 * t;
+    pp[g * nt * 8 + c] = d[0];
+    pp[g * nt * 8 + c + 1] = d[1];
+    pp[(g + 8) * nt * 8 + c] = d[2];
+    pp[(g + 8) * nt * 8 + c + 1] = d[3];
   }
   __syncthreads();
   for (int i = threadIdx.x; i < 16 * cols; i += kTinyThreads) {
     const int m = i / cols, c = i - m * cols;
     float v = 0.f;
-    for (int sp = 0; sp < split; ++sp) v += part[(sp * 16 + m) * cols + c];
+    for (int sp = 0; sp < split; ++sp) v += part[(static_cast<int64_t>(sp) * 16 + m) * nt * 8 + c];
     store(m, c, v);
   }
   __syncthreads();
@@ -124,25 +158,38 @@ __global__ void __launch_bounds__(kTinyThreads, 1) tiny_layer_kernel(TinyArgs a)
   griddep_launch_dependents();
   const int M = a.M, K = a.K, r = a.r, N = a.N;
   const TinyLayout L = tiny_layout(K, r, N);
-  float* xt = reinterpret_cast<float*>(smem + L.xt);
-  float* tt = reinterpret_cast<float*>(smem + L.tt);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs);
+  uint16_t* th = reinterpret_cast<uint16_t*>(smem + L.th);
+  uint16_t* tl = reinterpret_cast<uint16_t*>(smem + L.tl);
+  float* tf = reinterpret_cast<float*>(smem + L.t);
   float* part = reinterpret_cast<float*>(smem + L.part);
   uint8_t* as = smem + L.araw;
   uint8_t* bs = smem + L.braw;
   const uint32_t ao = stage_raw(as, a.A, static_cast<size_t>(K) * r * 2);
   const uint32_t bo = stage_raw(bs, a.B, static_cast<size_t>(r) * N * 2);
-  // X transposed to fp32 while A and B arrive (rows past M read as zero).
-  const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(a.X);
-  for (int i = threadIdx.x; i < 16 * K; i += kTinyThreads) {
-    const int k = i / 16, m = i - k * 16;
-    xt[i] = m < M ? __bfloat162float(X[static_cast<int64_t>(m) * K + k]) : 0.f;
+  // X into aligned bf16 rows while A and B arrive (zero past M and K).
+  const unsigned short* X = static_cast<const unsigned short*>(a.X);
+  for (int i = threadIdx.x; i < 16 * L.kp; i += kTinyThreads) {
+    const int m = i / L.kp, k = i - m * L.kp;
+    xs[i] = (m < M && k < K) ? X[static_cast<int64_t>(m) * K + k] : static_cast<unsigned short>(0);
   }
   cp_async_wait_all();
   __syncthreads();
-  // T = X·A, kept in fp32 (transposed for the second product).
-  tiny_product(xt, as, ao, r, K, r, part, [&](int m, int c, float v) { tt[c * 16 + m] = v; });
+  // T = X·A in fp32; then its bf16 hi and lo parts (zero past r) for the
+  // second product, so that T keeps about 16 bits.
+  tiny_mma_product(xs, nullptr, L.kp, as, ao, r, K, r, part,
+                   [&](int m, int c, float v) { tf[m * r + c] = v; });
+  for (int i = threadIdx.x; i < 16 * L.rp; i += kTinyThreads) {
+    const int m = i / L.rp, c = i - m * L.rp;
+    const float v = c < r ? tf[m * r + c] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    th[i] = __bfloat16_as_ushort(hi);
+    tl[i] = __bfloat16_as_ushort(lo);
+  }
+  __syncthreads();
   // Y = T·B + bias.
-  tiny_product(tt, bs, bo, N, r, N, part, [&](int m, int c, float v) {
+  tiny_mma_product(th, tl, L.rp, bs, bo, N, r, N, part, [&](int m, int c, float v) {
     if (m >= M) return;
     if (a.bias) v += __bfloat162float(a.bias[c]);
     const int64_t o = static_cast<int64_t>(m) * a.ldy + c;

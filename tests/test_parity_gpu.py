@@ -239,6 +239,41 @@ def test_fp32_output(lr, path, M, K, r, N):
     assert np.array_equal(f32_host(Z), np.broadcast_to(lrgen.bf16_to_f64(p["bias"]), (M, N)))
 
 
+@pytest.mark.parametrize("M,K,r,N", [(300, 333, 257, 517), (2048, 1024, 1741, 4096), (4, 4096, 333, 700)])
+def test_strided_operands_and_prepared_factors(lr, M, K, r, N):
+    """lr_linear_strided with padded row pitches for X, A, B and Y (bf16 and
+    fp32 outputs) against the oracle; with every prefill operand 32-byte
+    aligned at a 16-element pitch (factors in lr_factor_pitch buffers) the
+    call is one launch: no realignment copy."""
+    import torch
+    p = lrgen.lowrank_problem(M, K, r, N, seed=K + r, bias=True)
+    Yr = ref(p)
+
+    def padded(bits, pitch):
+        rows, cols = bits.shape
+        buf = torch.zeros((rows, pitch), dtype=torch.bfloat16, device="cuda")
+        buf[:, :cols] = to_dev(bits)
+        return buf[:, :cols]
+    X = padded(p["X"], lr.factor_pitch(K))
+    A = padded(p["A"], lr.factor_pitch(r))
+    B = padded(p["B"], lr.factor_pitch(N))
+    b = to_dev(p["bias"])
+    assert A.stride(0) == lr.factor_pitch(r) and lr.factor_pitch(r) % 64 == 0
+    Ybuf = torch.zeros((M, N + 3), dtype=torch.bfloat16, device="cuda")
+    n0 = lr.kernel_launch_count()
+    lr.lr_linear_strided(X, A, B, b, Y=Ybuf[:, :N])
+    torch.cuda.synchronize()
+    if M > 16:
+        assert lr.kernel_launch_count() - n0 == 1, "prepared operands must not be copied"
+    assert lr.last_device_status() == lr.LR_OK
+    compare(to_f64(Ybuf[:, :N].contiguous()), Yr, f"strided bf16 {M}x{K}x{r}x{N}")
+    assert np.all(to_f64(Ybuf[:, N:].contiguous()) == 0.0), "wrote past N"
+    Y32 = torch.zeros((M, N + 1), dtype=torch.float32, device="cuda")
+    lr.lr_linear_strided(X, A, B, b, Y=Y32[:, :N])
+    torch.cuda.synchronize()
+    compare(f32_host(Y32[:, :N]), Yr, f"strided fp32 {M}x{K}x{r}x{N}")
+
+
 # ---------------------------------------------------------------- edges
 def test_empty_and_degenerate(lr):
     import torch
