@@ -433,20 +433,26 @@ def layer_bench(lr, dev, peaks, n_int=14336):
         xs = {k: _dev_bits(v, dev) for k, v in layer["inputs"].items()}
         P = layer["projs"]
         packed = torch.empty((Ml, 2 * n_int), dtype=torch.bfloat16, device=dev)
-        entries, keep = [], []
-        for name, p in P.items():
-            A, B = _dev_bits(p["A"], dev), _dev_bits(p["B"], dev)
-            keep += [A, B]
-            e = dict(X=xs[p["x"]], A=A, B=B, K=p["K"], r=p["r"], N=p["N"])
-            if name in ("gate", "up"):
-                e["Y_ptr"] = packed.data_ptr() + (0 if name == "gate" else 2 * n_int)
-                e["ld_y"] = 2 * n_int
-            else:
-                Yp = torch.empty((Ml, p["N"]), dtype=torch.bfloat16, device=dev)
-                keep.append(Yp)
-                e["Y"] = Yp
-            entries.append(e)
-        tl = time_steps(lambda i: lr.lr_linear_group(entries, Ml), 20, 3) / 20
+        # At M = 1 the factors (~76 MB) would stay in L2 between steps: two
+        # copies of them alternate.
+        sets, keep = [], []
+        Ys = {name: torch.empty((Ml, p["N"]), dtype=torch.bfloat16, device=dev)
+              for name, p in P.items() if name not in ("gate", "up")}
+        for copy in range(2 if Ml == 1 else 1):
+            entries = []
+            for name, p in P.items():
+                A, B = _dev_bits(p["A"], dev), _dev_bits(p["B"], dev)
+                keep += [A, B]
+                e = dict(X=xs[p["x"]], A=A, B=B, K=p["K"], r=p["r"], N=p["N"])
+                if name in ("gate", "up"):
+                    e["Y_ptr"] = packed.data_ptr() + (0 if name == "gate" else 2 * n_int)
+                    e["ld_y"] = 2 * n_int
+                else:
+                    e["Y"] = Ys[name]
+                entries.append(e)
+            sets.append(entries)
+        step = lambda i: lr.lr_linear_group(sets[i % len(sets)], Ml)
+        tl = time_steps(step, 20, 3) / 20
         projs = [dict(K=p["K"], r=p["r"], N=p["N"], x=p["x"]) for p in P.values()]
         fl, by = acc.group_work(Ml, projs)
         dense_by = sum(acc.dense_bytes(Ml, p["K"], p["N"]) for p in P.values())
@@ -458,7 +464,43 @@ def layer_bench(lr, dev, peaks, n_int=14336):
                          "dense_roofline_us": droof.t_roof_s * 1e6,
                          "ranks": layer["ranks"], "keep_ratio": acc.keep_ratio(
                              [(p["K"], p["N"], p["r"]) for p in P.values()])}
+        if Ml == 1:
+            # Back-to-back eager calls at M = 1 wait on the host (building the
+            # call's table in Python); the same calls replayed from a CUDA
+            # graph give the device time.
+            tg = graph_us(step, 10, dev) * 1e-6
+            res["M1"].update({"graph_us": tg * 1e6, "frac_roofline_graph": roof.t_roof_s / tg,
+                              "launches_per_call": 1})
     return res
+
+
+def graph_us(fn, calls, dev):
+    """Device time per call of `calls` calls captured in one CUDA graph and
+    replayed three times (the library keeps a workspace per stream, so the
+    capture stream is warmed up first: nothing is allocated while capturing)."""
+    import torch
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        for i in range(3):
+            fn(i)
+    cs.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        for i in range(calls):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(3):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (3 * calls)
 
 
 def metric_name():
@@ -595,11 +637,13 @@ def run_ours(args):
                 def dstep(i, Xd=Xd, Ads=Ads, Bds=Bds, Yd=Yd, cps=cps):
                     lr.lr_linear(Xd, Ads[i % cps], Bds[i % cps], None, Y=Yd)
                 td = time_steps(dstep, 50, 5) / 50
+                tg = graph_us(dstep, 2 * cps, dev) * 1e-6
                 by = acc.algorithmic_bytes(dm, dk, dr, dn)
                 decode[f"{name}_M{dm}"] = {
                     "us": td * 1e6, "GB/s": by / td / 1e9,
                     "frac_hbm": by / td / 1e9 / peaks["hbm_gbs"],
                     "frac_hbm_spec": by / td / 1e9 / SPEC_PEAKS["hbm_gbs"],
+                    "graph_us": tg * 1e6, "frac_hbm_graph": by / tg / 1e9 / peaks["hbm_gbs"],
                     "dense_equiv_us_at_peak": acc.dense_bytes(dm, dk, dn) / (peaks["hbm_gbs"] * 1e9) * 1e6}
                 del Ads, Bds
 

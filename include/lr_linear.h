@@ -67,7 +67,8 @@ typedef enum {
  * K == 0 or r == 0: the sum is empty and Y = bias (or 0).
  *
  * Path: M <= 16 takes the decode kernels (bandwidth-bound streaming of A then
- * B, T kept in fp32); larger M takes the tcgen05 prefill path: one launch
+ * B, T kept in fp32; two launches, the second streaming B while the first
+ * finishes).  Larger M takes the tcgen05 prefill path: one launch
  * computes T = X·A (written once as bf16) and Y = T·B, GEMM2's tiles
  * waiting for GEMM1's rows inside the launch.  Neither path pads r on the
  * host.  Prefill operands whose rows do not start on 32-byte boundaries
@@ -167,8 +168,13 @@ typedef struct {
  * At M > 16 the group is one prefill launch when it fits the launch's tables
  * (at most 12 GEMMs: one per set of projections sharing X, plus one per
  * projection): projections with the same X pointer and K are one GEMM1 over
- * their A factors copied side by side; otherwise, and at M <= 16, the
- * projections run one by one.  FlashSVD v1.5's abstract describes the packed
+ * their A factors copied side by side.  At M <= 8 a group of at most 7
+ * projections, each with K, r, N > 0, is one persistent launch: every SM
+ * streams a slice of every projection's A, then of every B (rows of W
+ * through shared memory into mma.sync; T in fp32, multiplied as bf16
+ * hi + lo), each B block starting as soon as the blocks of T it needs are
+ * summed; results equal lr_linear's up to fp32 rounding (another kernel).
+ * Otherwise the projections run one by one.  FlashSVD v1.5's abstract describes the packed
  * execution of a layer's projections this mirrors (catalogue record of
  * arXiv 2605.08314).
  */
@@ -239,7 +245,10 @@ int lr_last_cuda_error(void);
  *   only; larger M returns LR_ERR_INVALID_ARG), 2 = force prefill, 3 = force
  *   prefill on single-SM tiles (the default prefill kernel), 4 = force prefill
  *   on CTA pairs (2-SM MMA, 256×256 tiles, GEMM1 and GEMM2 as two launches;
- *   M <= 128 still uses single SMs).
+ *   M <= 128 still uses single SMs), 5 = force decode on the two-launch
+ *   kernels, groups included (M <= 16 only), 6 = force decode, and for
+ *   M <= 8 on the streamed one-launch kernel that decode-size groups use
+ *   (M <= 16 only; see lr_linear_group).
  * lr_set_wait_limit_ns — time limit of every device-side bounded wait
  *   (default 2e9 ns); 0 restores the default.
  * lr_set_tile_n — column width of the prefill kernel's single-SM tiles:

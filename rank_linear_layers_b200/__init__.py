@@ -27,6 +27,7 @@ LR_ERR_NO_MEMORY = 5
 LR_ERR_INFEASIBLE = 6
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_PREFILL_1SM, PATH_PREFILL_PAIR = 0, 1, 2, 3, 4
+PATH_DECODE_TWO_LAUNCH, PATH_DECODE_STREAM = 5, 6
 
 # Every symbol include/lr_linear.h declares.
 EXPORTS = (

@@ -298,10 +298,190 @@ size_t ctr_bytes(int M, int64_t Kd, int64_t n, int sms) {
   return align_up(static_cast<size_t>(p.col_blocks) * 4, 256);
 }
 
+int64_t ceil_div(int64_t a, int64_t b);
+
+// One decode-size pair of jobs (T = X·A, then Y = T·B + bias) of the
+// streamed kernel, appended to `a`; its workspace areas are carved from
+// `zero` (zero at rest) and `scratch`, and its flags from `flags`.
+struct StreamPair {
+  const void *X, *A, *B, *bias;
+  void* Y;
+  int64_t K, r, N, ldy;
+  bool y_f32;
+  Pitch ld;
+};
+
+size_t stream_pair_zero(int M, const StreamPair& p) {
+  const int64_t n0 = ceil_div(p.r, stream_block_cols(p.r)), n1 = ceil_div(p.N, stream_block_cols(p.N));
+  return align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.r), 8) * 4, 256) +
+         align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.N), 8) * 4, 256) +
+         align_up(static_cast<size_t>(2 * n0 + n1) * 4, 256);
+}
+size_t stream_pair_scratch(int M, const StreamPair& p) {
+  return align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.r), 8) * 4, 256);
+}
+void stream_add_pair(StreamArgs& a, const StreamPair& p, char** zero, char** scratch) {
+  const int M = a.M;
+  const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(p.r), 8));
+  const int64_t ldn = static_cast<int64_t>(align_up(static_cast<size_t>(p.N), 8));
+  float* acc0 = reinterpret_cast<float*>(*zero);
+  *zero += align_up(static_cast<size_t>(M) * ldt * 4, 256);
+  float* acc1 = reinterpret_cast<float*>(*zero);
+  *zero += align_up(static_cast<size_t>(M) * ldn * 4, 256);
+  const int cb0 = stream_block_cols(p.r), cb1 = stream_block_cols(p.N);
+  const int64_t nb0 = ceil_div(p.r, cb0), nb1 = ceil_div(p.N, cb1);
+  unsigned int* cnt = reinterpret_cast<unsigned int*>(*zero);
+  unsigned int* ready = cnt + nb0 + nb1;
+  *zero += align_up(static_cast<size_t>(2 * nb0 + nb1) * 4, 256);
+  float* T = reinterpret_cast<float*>(*scratch);
+  *scratch += align_up(static_cast<size_t>(M) * ldt * 4, 256);
+
+  StreamJob& j0 = a.job[a.n_jobs];
+  j0 = StreamJob{};
+  j0.W = static_cast<const __nv_bfloat16*>(p.A);
+  j0.ldw = p.ld.a;
+  j0.w_lo = reinterpret_cast<uintptr_t>(p.A);
+  j0.w_hi = j0.w_lo + span_bytes(p.K, p.r, p.ld.a);
+  j0.K = static_cast<int>(p.K);
+  j0.N = static_cast<int>(p.r);
+  j0.cb = cb0;
+  j0.phase = 0;
+  j0.V = p.X;
+  j0.ldv = p.ld.x;
+  j0.src = -1;
+  j0.acc = acc0;
+  j0.ld_acc = ldt;
+  j0.cnt = cnt;
+  j0.ready = ready;
+  j0.out_f32 = T;
+  j0.ld_out = ldt;
+  j0.unit0 = a.units[0];
+  a.units[0] += p.K * p.r;
+  const int src = a.n_jobs++;
+
+  StreamJob& j1 = a.job[a.n_jobs++];
+  j1 = StreamJob{};
+  j1.W = static_cast<const __nv_bfloat16*>(p.B);
+  j1.ldw = p.ld.b;
+  j1.w_lo = reinterpret_cast<uintptr_t>(p.B);
+  j1.w_hi = j1.w_lo + span_bytes(p.r, p.N, p.ld.b);
+  j1.K = static_cast<int>(p.r);
+  j1.N = static_cast<int>(p.N);
+  j1.cb = cb1;
+  j1.phase = 1;
+  j1.V = T;
+  j1.ldv = ldt;
+  j1.src = src;
+  j1.acc = acc1;
+  j1.ld_acc = ldn;
+  j1.cnt = cnt + nb0;
+  j1.ready = nullptr;
+  if (p.y_f32)
+    j1.out_f32 = static_cast<float*>(p.Y);
+  else
+    j1.out_bf16 = static_cast<__nv_bfloat16*>(p.Y);
+  j1.ld_out = p.ldy;
+  j1.bias = static_cast<const __nv_bfloat16*>(p.bias);
+  j1.unit0 = a.units[1];
+  a.units[1] += p.r * p.N;
+  a.n_final += static_cast<int>(nb1);
+}
+
+// Every CTA's pieces for a set of job shapes, computed once on the host and
+// kept on the device (a few KB per set of shapes; the kernel reads its own
+// instead of computing them, which took its threads microseconds).  Kept
+// for the life of the process; a decode loop uses a handful of shapes.
+struct PieceTable {
+  StreamSeg* pieces = nullptr;
+  int* off = nullptr;
+};
+std::mutex g_piece_mu;
+std::map<std::vector<int64_t>, PieceTable> g_piece_tables;
+constexpr size_t kMaxPieceTables = 1024;
+
+// Attach the piece table of `a` (grid CTAs) to it: LR_OK, or
+// LR_ERR_UNSUPPORTED when a CTA's pieces exceed the kernel's list.
+lr_status stream_pieces(StreamArgs& a, int grid) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::vector<int64_t> key{dev, grid, a.n_jobs};
+  for (int j = 0; j < a.n_jobs; ++j)
+    key.insert(key.end(), {a.job[j].phase, a.job[j].K, a.job[j].N, a.job[j].cb});
+  std::lock_guard<std::mutex> lk(g_piece_mu);
+  auto it = g_piece_tables.find(key);
+  if (it == g_piece_tables.end()) {
+    std::vector<StreamSeg> all;
+    std::vector<int> off(static_cast<size_t>(grid) + 1, 0);
+    StreamSeg tmp[2 * kStreamMaxSegs];
+    for (int g = 0; g < grid; ++g) {
+      const int n = stream_segments(a, g, grid, tmp, 2 * kStreamMaxSegs);
+      if (n > 2 * kStreamMaxSegs) return LR_ERR_UNSUPPORTED;
+      all.insert(all.end(), tmp, tmp + n);
+      off[g + 1] = static_cast<int>(all.size());
+    }
+    if (g_piece_tables.size() >= kMaxPieceTables) {
+      // Too many shapes to keep: the CTAs compute their pieces themselves.
+      if (!std::all_of(off.begin() + 1, off.end(), [&, prev = 0](int o) mutable {
+            const bool ok = o - prev <= kStreamMaxSegs;
+            prev = o;
+            return ok;
+          }))
+        return LR_ERR_UNSUPPORTED;
+      a.pieces = nullptr;
+      a.piece_off = nullptr;
+      return LR_OK;
+    }
+    PieceTable t;
+    LR_CUDA(cudaMalloc(&t.pieces, std::max<size_t>(all.size(), 1) * sizeof(StreamSeg)));
+    LR_CUDA(cudaMalloc(&t.off, off.size() * sizeof(int)));
+    LR_CUDA(cudaMemcpy(t.pieces, all.data(), all.size() * sizeof(StreamSeg), cudaMemcpyHostToDevice));
+    LR_CUDA(cudaMemcpy(t.off, off.data(), off.size() * sizeof(int), cudaMemcpyHostToDevice));
+    it = g_piece_tables.emplace(key, t).first;
+  }
+  a.pieces = it->second.pieces;
+  a.piece_off = it->second.off;
+  return LR_OK;
+}
+
+// Decode-size pairs on the streamed kernel (M <= 8): one launch.
+lr_status run_stream(DeviceInfo* d, cudaStream_t stream, int M, const StreamPair* pairs, int n) {
+  size_t zneed = 256, sneed = 0;
+  for (int i = 0; i < n; ++i) {
+    zneed += stream_pair_zero(M, pairs[i]);
+    sneed += stream_pair_scratch(M, pairs[i]);
+  }
+  char *zero = nullptr, *scratch = nullptr;
+  lr_status st = workspace(stream, zneed, sneed, &zero, &scratch);
+  if (st != LR_OK) return st;
+  StreamArgs a{};
+  a.M = M;
+  a.done = reinterpret_cast<unsigned int*>(zero);
+  zero += 256;
+  for (int i = 0; i < n; ++i) stream_add_pair(a, pairs[i], &zero, &scratch);
+  a.w_early = 1;
+  a.wait = wait_ctl(d);
+  st = stream_pieces(a, d->sms);
+  if (st != LR_OK) return st;
+  return launched(launch_stream(a, d->sms, stream, false));
+}
+
+// A single decode call takes the two-launch skinny kernels, or with path 6
+// (M <= 8) the streamed one-launch kernel.  (Measured on B200 at the
+// Llama-3-8B MLP shapes, M = 1: 32 µs two-launch, 59 µs streamed; the
+// streamed kernel pays ~5 µs at each piece boundary and waits for the
+// slowest CTA's phase 0.  It is the decode group's kernel, where one launch
+// replaces fourteen.)
+bool use_stream(int64_t M) { return g_path.load() == 6 && M <= 8; }
+
 lr_status run_decode(DeviceInfo* d, cudaStream_t stream, const void* X, const void* A,
                      const void* B, const void* bias, void* Y, int64_t M, int64_t K, int64_t r,
                      int64_t N, int64_t ldy, bool y_f32, Pitch ld) {
   const int m = static_cast<int>(M);
+  if (use_stream(M)) {
+    const StreamPair p{X, A, B, bias, Y, K, r, N, ldy, y_f32, ld};
+    lr_status st = run_stream(d, stream, m, &p, 1);
+    if (st != LR_ERR_UNSUPPORTED) return st;
+  }
   const size_t acc1 = acc_bytes(m, r), acc2 = acc_bytes(m, N);
   const size_t c1 = ctr_bytes(m, K, r, d->sms), c2 = ctr_bytes(m, r, N, d->sms);
   const int64_t ldt = static_cast<int64_t>(align_up(static_cast<size_t>(r), 4));
@@ -488,17 +668,37 @@ double epilogue_us(int bn) { return 0.6 + 1.0 * bn / 256.0; }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// K splits of a GEMM with `tiles` output tiles and `nkb` k blocks: a GEMM
+// with too few tiles to fill half the SMs and a long K loop (GEMM1 at small
+// ranks) splits K, up to one split per 8 k blocks, as many as fill the SMs.
+// Returns the k blocks per split; *splits receives the split count.
+int split_plan(int64_t tiles, int nkb, int sms, int* splits) {
+  int s = 1;
+  if (g_split_k.load() && tiles * 2 <= sms && nkb >= 16)
+    s = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({nkb / 8, sms / tiles, 16})));
+  const int per = static_cast<int>(ceil_div(nkb, s));
+  *splits = static_cast<int>(ceil_div(nkb, per));
+  return per;
+}
+
 // Simulate the static round-robin schedule of the chain kernel.
 // A k block of a problem whose operand a has two parts issues twice the
-// tensor-core work of its tile width.
+// tensor-core work of its tile width.  The splits of a split tile are
+// consecutive items; each adds fp32 partial sums to the workspace (costed
+// as two epilogues of its width) and the tile is done one epilogue after
+// its last split.
 double kblock_cost(const ChainProblem& P, int bn) {
   return kblock_us(P.map_a_lo >= 0 ? 2 * bn : bn);
 }
 
 double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
   int64_t total = 0;
-  for (int i = 0; i < a.n_prob; ++i)
-    total += ceil_div(a.p[i].Mr, kGemmBM) * ceil_div(a.p[i].Nc, bn[i]);
+  std::vector<int> splits(static_cast<size_t>(a.n_prob)), per(static_cast<size_t>(a.n_prob));
+  for (int i = 0; i < a.n_prob; ++i) {
+    const int64_t tiles = ceil_div(a.p[i].Mr, kGemmBM) * ceil_div(a.p[i].Nc, bn[i]);
+    per[i] = split_plan(tiles, static_cast<int>(ceil_div(a.p[i].Kc, kGemmBK)), sms, &splits[i]);
+    total += tiles * splits[i];
+  }
   const int64_t G = std::max<int64_t>(1, std::min<int64_t>(total, sms));
   std::vector<double> t(static_cast<size_t>(G), 0.0);
   std::map<int, std::vector<double>> ready;
@@ -507,7 +707,8 @@ double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
   for (int i = 0; i < a.n_prob; ++i) {
     const ChainProblem& P = a.p[i];
     const int64_t tm = ceil_div(P.Mr, kGemmBM), tn = ceil_div(P.Nc, bn[i]);
-    const double dur = static_cast<double>(ceil_div(P.Kc, kGemmBK)) * kblock_cost(P, bn[i]) + 0.15;
+    const int nkb = static_cast<int>(ceil_div(P.Kc, kGemmBK));
+    const double epi = epilogue_us(bn[i]);
     std::vector<double>* sig = nullptr;
     const std::vector<double>* wait = nullptr;
     if (P.signal_group >= 0) {
@@ -518,15 +719,20 @@ double simulate_chain(const ChainArgs& a, const std::vector<int>& bn, int sms) {
       auto it = ready.find(P.wait_group);
       if (it != ready.end()) wait = &it->second;
     }
-    for (int64_t l = 0; l < tm * tn; ++l, ++idx) {
-      double& tc = t[static_cast<size_t>(idx % G)];
+    for (int64_t l = 0; l < tm * tn; ++l) {
       const int64_t m = l / tn;
-      double start = tc;
-      if (wait && m < static_cast<int64_t>(wait->size())) start = std::max(start, (*wait)[m]);
-      tc = start + dur;
-      if (sig) (*sig)[m] = std::max((*sig)[m], tc + epilogue_us(bn[i]));
+      double done = 0.0;
+      for (int s = 0; s < splits[i]; ++s, ++idx) {
+        double& tc = t[static_cast<size_t>(idx % G)];
+        double start = tc;
+        if (wait && m < static_cast<int64_t>(wait->size())) start = std::max(start, (*wait)[m]);
+        const int kb = std::min(per[i], nkb - s * per[i]);
+        tc = start + kb * kblock_cost(P, bn[i]) + 0.15 + (splits[i] > 1 ? 2.0 * epi : 0.0);
+        done = std::max(done, tc);
+      }
+      if (sig) (*sig)[m] = std::max((*sig)[m], done + epi);
     }
-    tail = epilogue_us(bn[i]);
+    tail = epi;
   }
   return *std::max_element(t.begin(), t.end()) + tail;
 }
@@ -539,7 +745,7 @@ std::map<std::vector<int64_t>, std::vector<int>> g_plans;
 // by coordinate descent from the widest tiles.
 std::vector<int> plan_chain(const ChainArgs& a, int sms) {
   const int forced = g_tile_n.load();
-  std::vector<int64_t> key{sms, forced};
+  std::vector<int64_t> key{sms, forced, g_split_k.load()};
   for (int i = 0; i < a.n_prob; ++i) {
     const ChainProblem& P = a.p[i];
     key.insert(key.end(), {P.Mr, P.Nc, P.Kc, P.wait_group, P.signal_group, P.map_a_lo >= 0});
@@ -605,9 +811,7 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
     ChainProblem& P = a.p[i];
     if (P.signal_group >= 0) groups = std::max(groups, P.signal_group + 1);
   }
-  // Split K for a GEMM with too few tiles to fill half the SMs and a long
-  // K loop (GEMM1 at small ranks): up to one split per 8 k blocks, as many
-  // as fill the SMs.
+  // K splits: split_plan.
   int64_t split_floats = 0;
   for (int i = 0; i < a.n_prob; ++i) {
     ChainProblem& P = a.p[i];
@@ -615,12 +819,8 @@ lr_status run_chain(DeviceInfo* d, cudaStream_t stream, ChainBuild& cb) {
     P.tiles_m = static_cast<int>(ceil_div(P.Mr, kGemmBM));
     P.tiles_n = static_cast<int>(ceil_div(P.Nc, P.bn));
     const int64_t tiles = static_cast<int64_t>(P.tiles_m) * P.tiles_n;
-    const int nkb = static_cast<int>(ceil_div(P.Kc, kGemmBK));
-    int splits = 1;
-    if (g_split_k.load() && tiles * 2 <= d->sms && nkb >= 16)
-      splits = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({nkb / 8, d->sms / tiles, 16})));
-    P.kb_per_split = static_cast<int>(ceil_div(nkb, splits));
-    P.splits = static_cast<int>(ceil_div(nkb, P.kb_per_split));
+    P.kb_per_split =
+        split_plan(tiles, static_cast<int>(ceil_div(P.Kc, kGemmBK)), d->sms, &P.splits);
     P.split_group = -1;
     if (P.splits > 1) {
       P.split_group = groups++;
@@ -843,7 +1043,7 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
   lr_status st = validate(X, A, B, bias, Y, M, K, r, N, ldy, y_f32, ld);
   if (st != LR_OK) return st;
   const int path = g_path.load();
-  if (path == 1 && M > 16) return LR_ERR_INVALID_ARG;
+  if ((path == 1 || path == 5 || path == 6) && M > 16) return LR_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return LR_OK;
   DeviceInfo* d = nullptr;
   int dev = 0;
@@ -872,7 +1072,7 @@ lr_status run_linear(const void* X, const void* A, const void* B, const void* bi
     t.y_f32 = y_f32 ? 1 : 0;
     return launched(launch_tiny(t, stream));
   }
-  const bool decode = (path == 1) || (path == 0 && M <= 16);
+  const bool decode = (path == 1) || (path == 5) || (path == 6) || (path == 0 && M <= 16);
   if (decode) {
     note_call(stream, false, Y, ybytes);
     return run_decode(d, stream, X, A, B, bias, Y, M, K, r, N, ldy, y_f32, ld);
@@ -1145,13 +1345,37 @@ lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* str
   }
   // Prefill sizes: the whole group in one chain launch (see run_group_prefill).
   const int path = g_path.load();
-  if (M > 16 && path != 1 && path != 4 && n_proj > 0) {
+  if (M > 16 && path != 1 && path != 4 && path != 5 && path != 6 && n_proj > 0) {
     DeviceInfo* d = nullptr;
     int dev = 0;
     lr_status st = device_info(&d, &dev);
     if (st != LR_OK) return st;
     st = run_group_prefill(d, static_cast<cudaStream_t>(stream), projs, n_proj, M);
     if (st != LR_ERR_UNSUPPORTED) return st;
+  }
+  // Decode sizes (M <= 8): the whole group in one streamed launch, when
+  // every projection has work (K, r, N > 0) and the group fits the launch's
+  // table (at most kStreamMaxJobs / 2 projections).
+  if (M > 0 && M <= 8 && (path == 0 || path == 6) && n_proj > 0 &&
+      n_proj <= kStreamMaxJobs / 2) {
+    bool all = true;
+    for (int i = 0; i < n_proj; ++i) all = all && projs[i].K > 0 && projs[i].r > 0 && projs[i].N > 0;
+    if (all) {
+      DeviceInfo* d = nullptr;
+      int dev = 0;
+      lr_status st = device_info(&d, &dev);
+      if (st != LR_OK) return st;
+      StreamPair pairs[kStreamMaxJobs / 2];
+      for (int i = 0; i < n_proj; ++i) {
+        const lr_proj& p = projs[i];
+        pairs[i] = StreamPair{p.X, p.A, p.B, p.bias, p.Y, p.K, p.r, p.N, p.ld_y, p.y_f32 != 0,
+                              Pitch{p.K, p.r, p.N}};
+        note_call(static_cast<cudaStream_t>(stream), false, p.Y,
+                  span_bytes(M, p.N, p.ld_y) * (p.y_f32 ? 2 : 1));
+      }
+      st = run_stream(d, static_cast<cudaStream_t>(stream), static_cast<int>(M), pairs, n_proj);
+      if (st != LR_ERR_UNSUPPORTED) return st;
+    }
   }
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];
@@ -1226,7 +1450,7 @@ lr_status lr_dense(const void* X, const void* W, const void* bias, void* Y, int6
     return launched(launch_fill_bias(Y, false, N, M, N, static_cast<const __nv_bfloat16*>(bias),
                                      stream));
   const int path = g_path.load();
-  const bool decode = (path == 1) || (path == 0 && M <= 16);
+  const bool decode = (path == 1) || (path == 5) || (path == 6) || (path == 0 && M <= 16);
   if (decode) {
     if (M > 16) return LR_ERR_INVALID_ARG;
     const int m = static_cast<int>(M);
@@ -1304,7 +1528,7 @@ const char* lr_status_string(lr_status s) {
 int lr_last_cuda_error(void) { return g_last_cuda_error; }
 
 lr_status lr_set_path(int path) {
-  if (path < 0 || path > 4) return LR_ERR_INVALID_ARG;
+  if (path < 0 || path > 6) return LR_ERR_INVALID_ARG;
   g_path.store(path);
   return LR_OK;
 }

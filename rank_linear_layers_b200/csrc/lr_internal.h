@@ -28,6 +28,142 @@ cudaError_t ensure_max_smem(const void* kernel, int bytes);
 // The time limit of device-side bounded waits (lr_set_wait_limit_ns).
 unsigned long long wait_limit_ns();
 
+// ------------------------------------------------------- streamed decode
+// out[m, n] = sum_k V[m, k] · W[k, n] (m < M <= 8) for several "jobs" in
+// one persistent launch (one CTA per SM).  A job's W is cut into column
+// blocks of cb <= 248 columns; every CTA takes one contiguous slice of each
+// phase's (block, row) units, weighted by block width, and streams its rows
+// of W through shared memory into the tensor cores.  Phase-0 jobs read a bf16 V; a phase-1 job reads
+// as V the fp32 result of phase-0 job `src`, block by block as each block of
+// it is finished (a flag per block), so its W stream starts before phase 0
+// ends.  The CTA that finishes the last phase-1 block clears the flags: the
+// workspace is zero again when the launch ends, and the launch can be
+// replayed from a CUDA graph.
+constexpr int kStreamMaxJobs = 14;
+constexpr int kStreamMaxSegs = 64;  // (job, block, row range) pieces per CTA
+
+struct StreamSeg {
+  int job, b, k0, k1;      // rows [k0, k1) of block b of job `job`
+};
+
+struct StreamJob {
+  const __nv_bfloat16* W;  // [K, ldw] bf16
+  int64_t ldw;
+  uintptr_t w_lo, w_hi;    // byte extent of W's rows
+  int K, N;                // rows and columns of W
+  int cb;                  // columns per block: a multiple of 8, at most 248
+  int phase;               // 0 or 1
+  const void* V;           // [M, ldv]: bf16 (phase 0) or fp32 (phase 1)
+  int64_t ldv;
+  int src;                 // phase 1: the job whose result V is
+  float* acc;              // [M, ld_acc] fp32 partial sums, zero at rest
+  int64_t ld_acc;
+  unsigned int* cnt;       // [blocks] rows added so far, zero at rest
+  unsigned int* ready;     // [blocks] 1 once the block is finished (phase 0), zero at rest
+  float* out_f32;          // fp32 result [M, ld_out], or null
+  __nv_bfloat16* out_bf16; // bf16 result [M, ld_out], or null
+  int64_t ld_out;
+  const __nv_bfloat16* bias;  // [N] added to the result, or null
+  int64_t unit0;           // first unit of the job within its phase (unit = one element of W)
+};
+
+struct StreamArgs {
+  StreamJob job[kStreamMaxJobs];
+  int n_jobs;
+  int M;
+  unsigned int* done;      // phase-1 blocks finished so far, zero at rest
+  int n_final;             // phase-1 blocks in all
+  // Each CTA's pieces (stream_segments), computed once per set of job
+  // shapes: CTA g's are pieces[piece_off[g] .. piece_off[g + 1]).  Null:
+  // the CTAs compute their own.
+  const StreamSeg* pieces;
+  const int* piece_off;
+  int w_early;             // W may be read before the previous launch on the stream ends
+  int64_t units[2];        // units of each phase
+  WaitCtl wait;
+};
+
+
+
+// floor(x / w) for 0 <= x < 2^53, w > 0.  On the device through a double
+// division and an exact correction (a 64-bit integer division is a long
+// software routine there).
+__host__ __device__ inline int64_t stream_div(int64_t x, int64_t w) {
+#ifdef __CUDA_ARCH__
+  int64_t q = static_cast<int64_t>(static_cast<double>(x) / static_cast<double>(w));
+  while (q > 0 && q * w > x) --q;
+  while ((q + 1) * w <= x) ++q;
+  return q;
+#else
+  return x / w;
+#endif
+}
+
+__host__ __device__ inline int64_t stream_cdiv_clamp(int64_t x, int64_t w, int64_t hi) {
+  if (x <= 0) return 0;
+  const int64_t q = stream_div(x + w - 1, w);
+  return q < hi ? q : hi;
+}
+
+// The pieces CTA g of G streams, phase 0 first: in each phase the units
+// [U·g/G, U·(g+1)/G) of the phase's jobs laid end to end, a job's units in
+// block order and, within a block, row by row (a row of block b is width(b)
+// units).  A row belongs to the CTA whose range holds its first unit.
+// Writes at most `cap` pieces; returns how many there are.
+__host__ __device__ inline int stream_segments(const StreamArgs& a, int g, int G, StreamSeg* out,
+                                               int cap) {
+  int n = 0;
+  for (int ph = 0; ph < 2; ++ph) {
+    const int64_t U = a.units[ph];
+    if (U <= 0) continue;
+    const int64_t lo = U * g / G, hi = U * (g + 1) / G;
+    for (int j = 0; j < a.n_jobs; ++j) {
+      const StreamJob& J = a.job[j];
+      if (J.phase != ph) continue;
+      const int64_t K = J.K, N = J.N, cb = J.cb;
+      if (J.unit0 >= hi || J.unit0 + K * N <= lo) continue;
+      const int64_t nb = (N + cb - 1) / cb;
+      for (int64_t b = 0; b < nb; ++b) {
+        const int64_t wb = (N - b * cb) < cb ? (N - b * cb) : cb;
+        const int64_t base = J.unit0 + b * K * cb;
+        const int64_t k0 = stream_cdiv_clamp(lo - base, wb, K);
+        const int64_t k1 = stream_cdiv_clamp(hi - base, wb, K);
+        if (k0 < k1) {
+          if (n < cap) out[n] = StreamSeg{j, static_cast<int>(b), static_cast<int>(k0),
+                                          static_cast<int>(k1)};
+          ++n;
+        }
+      }
+    }
+  }
+  return n;
+}
+
+// The piece of block b of job j that CTA g of G takes (k0 == k1: none); the
+// same rule as stream_segments, for one block.
+__host__ __device__ inline StreamSeg stream_piece(const StreamArgs& a, int j, int64_t b, int g,
+                                                  int G) {
+  const StreamJob& J = a.job[j];
+  const int64_t U = a.units[J.phase];
+  const int64_t lo = stream_div(U * g, G), hi = stream_div(U * (g + 1), G);
+  const int64_t K = J.K, N = J.N, cb = J.cb;
+  const int64_t wb = (N - b * cb) < cb ? (N - b * cb) : cb;
+  const int64_t base = J.unit0 + b * K * cb;
+  const int64_t k0 = stream_cdiv_clamp(lo - base, wb, K);
+  const int64_t k1 = stream_cdiv_clamp(hi - base, wb, K);
+  return StreamSeg{j, static_cast<int>(b), static_cast<int>(k0), static_cast<int>(k1)};
+}
+
+// Column block width for an output of n columns: the fewest blocks of at
+// most 248 columns, of equal width rounded up to a multiple of 8 (a row's
+// window of up to 248 + 7 columns is 32 granules of 16 bytes).
+inline int stream_block_cols(int64_t n) {
+  const int64_t nb = (n + 247) / 248;
+  return static_cast<int>(((n + nb - 1) / nb + 7) / 8 * 8);
+}
+
+cudaError_t launch_stream(const StreamArgs& a, int grid, cudaStream_t stream, bool dependent);
+
 // ------------------------------------------------------------------ decode
 // out[m, n] = sum_k V[m, k] · W[k, n] for m < M (M <= 16), W a bf16 [Kd, Nd]
 // row-major matrix with row stride ldw.  Split over column blocks (grid.x)
