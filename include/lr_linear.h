@@ -157,6 +157,13 @@ typedef struct {
   int64_t r;
   int64_t N;
   int32_t y_f32;
+  /* 0: none.  j + 1: projection j of the same group is this one's gate, and
+   * this projection's Y receives silu(G) * P instead of P, where P is its
+   * own product (X·A·B + bias, fp32) and G the gate's Y as stored (bf16 or
+   * fp32); silu(g) = g / (1 + e^-g).  The gated MLP's SiLU(gate) ⊙ up on the
+   * way to the down projection.  The gate must have the same N and no gate
+   * of its own. */
+  int32_t silu_gate;
 } lr_proj;
 
 /*
@@ -177,6 +184,13 @@ typedef struct {
  * Otherwise the projections run one by one.  FlashSVD v1.5's abstract describes the packed
  * execution of a layer's projections this mirrors (catalogue record of
  * arXiv 2605.08314).
+ * silu_gate: at M <= 8 the product silu(G) * P is formed where the
+ * streamed launch writes the up projection's blocks (each block waits,
+ * bounded, for the same block of the gate); on the other paths P goes to a
+ * library-owned fp32 buffer and one elementwise launch forms it.  Either
+ * way P is not rounded before the product; the result is rounded once.
+ * A projection with silu_gate, or one that is a gate, must not share Y
+ * memory with the inputs of any projection (checked like every Y).
  */
 lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream);
 

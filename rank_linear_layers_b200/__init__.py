@@ -54,7 +54,7 @@ class LrProj(ctypes.Structure):
         ("X", ctypes.c_void_p), ("K", ctypes.c_int64), ("A", ctypes.c_void_p),
         ("B", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("Y", ctypes.c_void_p),
         ("ld_y", ctypes.c_int64), ("r", ctypes.c_int64), ("N", ctypes.c_int64),
-        ("y_f32", ctypes.c_int32),
+        ("y_f32", ctypes.c_int32), ("silu_gate", ctypes.c_int32),
     ]
 
 
@@ -241,6 +241,8 @@ def lr_linear_group(projs: Sequence[dict], M: int, stream=None):
     entries are tensors) and y_f32 (Y is fp32; default: inferred from a Y
     tensor's dtype, else bf16).  Y may be a view into a packed buffer: pass
     the element pointer and ld_y explicitly via ``Y_ptr`` / ``ld_y``.
+    ``silu_gate``: the list index of this projection's gate (its Y becomes
+    silu(Y_gate) * its own product), or None.
     """
     import torch
     arr = (LrProj * max(1, len(projs)))()
@@ -255,7 +257,8 @@ def lr_linear_group(projs: Sequence[dict], M: int, stream=None):
                         _ptr(A) if hasattr(A, "data_ptr") else A,
                         _ptr(B) if hasattr(B, "data_ptr") else B,
                         _ptr(p.get("bias")) if hasattr(p.get("bias"), "data_ptr") else p.get("bias"),
-                        y_ptr, p.get("ld_y", N), r, N, 1 if y32 else 0)
+                        y_ptr, p.get("ld_y", N), r, N, 1 if y32 else 0,
+                        0 if p.get("silu_gate") is None else int(p["silu_gate"]) + 1)
     _check(lib().lr_linear_group(arr, len(projs), M, _stream_ptr(stream)), "lr_linear_group")
 
 

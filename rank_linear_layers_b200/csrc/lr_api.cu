@@ -55,6 +55,10 @@ struct Workspace {
   // calls (a call's repack may overlap the previous call's chain launch).
   char* rp_area[2] = {nullptr, nullptr};
   size_t rp_cap = 0;
+  // fp32 products of gated group projections (paths that do not fuse the
+  // gate's product).
+  float* act = nullptr;
+  size_t act_cap = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
@@ -309,13 +313,14 @@ struct StreamPair {
   int64_t K, r, N, ldy;
   bool y_f32;
   Pitch ld;
+  int gate = -1;  // index (in the same array) of the pair gating this one's output
 };
 
 size_t stream_pair_zero(int M, const StreamPair& p) {
   const int64_t n0 = ceil_div(p.r, stream_block_cols(p.r)), n1 = ceil_div(p.N, stream_block_cols(p.N));
   return align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.r), 8) * 4, 256) +
          align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.N), 8) * 4, 256) +
-         align_up(static_cast<size_t>(2 * n0 + n1) * 4, 256);
+         align_up(static_cast<size_t>(2 * n0 + 2 * n1) * 4, 256);
 }
 size_t stream_pair_scratch(int M, const StreamPair& p) {
   return align_up(static_cast<size_t>(M) * align_up(static_cast<size_t>(p.r), 8) * 4, 256);
@@ -332,7 +337,8 @@ void stream_add_pair(StreamArgs& a, const StreamPair& p, char** zero, char** scr
   const int64_t nb0 = ceil_div(p.r, cb0), nb1 = ceil_div(p.N, cb1);
   unsigned int* cnt = reinterpret_cast<unsigned int*>(*zero);
   unsigned int* ready = cnt + nb0 + nb1;
-  *zero += align_up(static_cast<size_t>(2 * nb0 + nb1) * 4, 256);
+  unsigned int* fin = ready + nb0;
+  *zero += align_up(static_cast<size_t>(2 * nb0 + 2 * nb1) * 4, 256);
   float* T = reinterpret_cast<float*>(*scratch);
   *scratch += align_up(static_cast<size_t>(M) * ldt * 4, 256);
 
@@ -383,6 +389,7 @@ void stream_add_pair(StreamArgs& a, const StreamPair& p, char** zero, char** scr
   j1.ld_out = p.ldy;
   j1.bias = static_cast<const __nv_bfloat16*>(p.bias);
   j1.unit0 = a.units[1];
+  j1.fin = fin;
   a.units[1] += p.r * p.N;
   a.n_final += static_cast<int>(nb1);
 }
@@ -457,7 +464,27 @@ lr_status run_stream(DeviceInfo* d, cudaStream_t stream, int M, const StreamPair
   a.M = M;
   a.done = reinterpret_cast<unsigned int*>(zero);
   zero += 256;
-  for (int i = 0; i < n; ++i) stream_add_pair(a, pairs[i], &zero, &scratch);
+  // Gates first: a CTA's phase-1 pieces run in job order, so a gated block
+  // never waits for a gate block that the same CTA has yet to stream.
+  std::vector<int> order, job1(static_cast<size_t>(n), -1);
+  for (int i = 0; i < n; ++i)
+    if (pairs[i].gate < 0) order.push_back(i);
+  for (int i = 0; i < n; ++i)
+    if (pairs[i].gate >= 0) order.push_back(i);
+  for (int i : order) {
+    stream_add_pair(a, pairs[i], &zero, &scratch);
+    job1[static_cast<size_t>(i)] = a.n_jobs - 1;
+  }
+  for (int i = 0; i < n; ++i) {
+    const int g = pairs[i].gate;
+    if (g < 0) continue;
+    StreamJob& J = a.job[job1[static_cast<size_t>(i)]];
+    const StreamJob& Gj = a.job[job1[static_cast<size_t>(g)]];
+    J.gate_y = pairs[g].Y;
+    J.gate_ld = pairs[g].ldy;
+    J.gate_f32 = pairs[g].y_f32 ? 1 : 0;
+    J.gate_fin = Gj.fin;
+  }
   a.w_early = 1;
   a.wait = wait_ctl(d);
   st = stream_pieces(a, d->sms);
@@ -1323,8 +1350,38 @@ int64_t lr_factor_pitch(int64_t cols) {
   return (cols + kPitchElems - 1) / kPitchElems * kPitchElems;
 }
 
+// The area for the fp32 products of a group's gated projections on
+// `stream` (`bytes`, grown on demand).
+lr_status act_area(cudaStream_t stream, size_t bytes, float** out) {
+  int dev = 0;
+  LR_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  if (bytes > w.act_cap) {
+    if (w.act) {
+      LR_CUDA(cudaStreamSynchronize(stream));
+      LR_CUDA(cudaFree(w.act));
+      w.act = nullptr;
+      w.act_cap = 0;
+    }
+    const size_t cap = align_up(bytes + bytes / 4, 1 << 20);
+    LR_CUDA(cudaMalloc(&w.act, cap));
+    w.act_cap = cap;
+  }
+  *out = w.act;
+  return LR_OK;
+}
+
 lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* stream) {
   if (n_proj < 0 || (n_proj > 0 && !projs) || M < 0) return LR_ERR_INVALID_ARG;
+  bool gated = false;
+  for (int i = 0; i < n_proj; ++i) {
+    const int g = projs[i].silu_gate - 1;
+    if (g == -1) continue;
+    if (g < 0 || g >= n_proj || g == i || projs[g].silu_gate != 0 || projs[g].N != projs[i].N)
+      return LR_ERR_INVALID_ARG;
+    gated = true;
+  }
   // Validate everything before the first launch, including Y overlaps.
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];
@@ -1343,24 +1400,18 @@ lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* str
       }
     }
   }
-  // Prefill sizes: the whole group in one chain launch (see run_group_prefill).
   const int path = g_path.load();
-  if (M > 16 && path != 1 && path != 4 && path != 5 && path != 6 && n_proj > 0) {
-    DeviceInfo* d = nullptr;
-    int dev = 0;
-    lr_status st = device_info(&d, &dev);
-    if (st != LR_OK) return st;
-    st = run_group_prefill(d, static_cast<cudaStream_t>(stream), projs, n_proj, M);
-    if (st != LR_ERR_UNSUPPORTED) return st;
-  }
+  const bool streamed = M > 0 && M <= 8 && (path == 0 || path == 6) && n_proj > 0 &&
+                        n_proj <= kStreamMaxJobs / 2;
+  bool all_work = true;
+  for (int i = 0; i < n_proj; ++i)
+    all_work = all_work && projs[i].K > 0 && projs[i].r > 0 && projs[i].N > 0;
   // Decode sizes (M <= 8): the whole group in one streamed launch, when
   // every projection has work (K, r, N > 0) and the group fits the launch's
-  // table (at most kStreamMaxJobs / 2 projections).
-  if (M > 0 && M <= 8 && (path == 0 || path == 6) && n_proj > 0 &&
-      n_proj <= kStreamMaxJobs / 2) {
-    bool all = true;
-    for (int i = 0; i < n_proj; ++i) all = all && projs[i].K > 0 && projs[i].r > 0 && projs[i].N > 0;
-    if (all) {
+  // table (at most kStreamMaxJobs / 2 projections); gated outputs are formed
+  // there.
+  if (streamed) {
+    if (all_work) {
       DeviceInfo* d = nullptr;
       int dev = 0;
       lr_status st = device_info(&d, &dev);
@@ -1369,13 +1420,56 @@ lr_status lr_linear_group(const lr_proj* projs, int n_proj, int64_t M, void* str
       for (int i = 0; i < n_proj; ++i) {
         const lr_proj& p = projs[i];
         pairs[i] = StreamPair{p.X, p.A, p.B, p.bias, p.Y, p.K, p.r, p.N, p.ld_y, p.y_f32 != 0,
-                              Pitch{p.K, p.r, p.N}};
+                              Pitch{p.K, p.r, p.N}, p.silu_gate - 1};
         note_call(static_cast<cudaStream_t>(stream), false, p.Y,
                   span_bytes(M, p.N, p.ld_y) * (p.y_f32 ? 2 : 1));
       }
       st = run_stream(d, static_cast<cudaStream_t>(stream), static_cast<int>(M), pairs, n_proj);
       if (st != LR_ERR_UNSUPPORTED) return st;
     }
+  }
+  if (gated) {
+    // Gated outputs without the fused path: the gated projections' products
+    // go to an fp32 area, the group runs as usual, then one elementwise
+    // launch per gated projection forms silu(G) · P.
+    if (M == 0) return LR_OK;
+    size_t need = 0;
+    for (int i = 0; i < n_proj; ++i)
+      if (projs[i].silu_gate) need += align_up(static_cast<size_t>(M * projs[i].N) * 4, 256);
+    float* area = nullptr;
+    lr_status st = act_area(static_cast<cudaStream_t>(stream), need, &area);
+    if (st != LR_OK) return st;
+    std::vector<lr_proj> q(projs, projs + n_proj);
+    std::vector<float*> prod(static_cast<size_t>(n_proj), nullptr);
+    for (int i = 0; i < n_proj; ++i) {
+      if (!projs[i].silu_gate) continue;
+      prod[i] = area;
+      area += align_up(static_cast<size_t>(M * projs[i].N) * 4, 256) / 4;
+      q[i].Y = prod[i];
+      q[i].ld_y = projs[i].N;
+      q[i].y_f32 = 1;
+      q[i].silu_gate = 0;
+    }
+    st = lr_linear_group(q.data(), n_proj, M, stream);
+    if (st != LR_OK) return st;
+    for (int i = 0; i < n_proj; ++i) {
+      if (!projs[i].silu_gate) continue;
+      const lr_proj& g = projs[projs[i].silu_gate - 1];
+      st = launched(launch_silu_mul(g.Y, g.ld_y, g.y_f32 != 0, prod[i], projs[i].Y,
+                                    projs[i].ld_y, projs[i].y_f32 != 0, M, projs[i].N,
+                                    static_cast<cudaStream_t>(stream)));
+      if (st != LR_OK) return st;
+    }
+    return LR_OK;
+  }
+  // Prefill sizes: the whole group in one chain launch (see run_group_prefill).
+  if (M > 16 && path != 1 && path != 4 && path != 5 && path != 6 && n_proj > 0) {
+    DeviceInfo* d = nullptr;
+    int dev = 0;
+    lr_status st = device_info(&d, &dev);
+    if (st != LR_OK) return st;
+    st = run_group_prefill(d, static_cast<cudaStream_t>(stream), projs, n_proj, M);
+    if (st != LR_ERR_UNSUPPORTED) return st;
   }
   for (int i = 0; i < n_proj; ++i) {
     const lr_proj& p = projs[i];

@@ -65,6 +65,13 @@ struct StreamJob {
   int64_t ld_out;
   const __nv_bfloat16* bias;  // [N] added to the result, or null
   int64_t unit0;           // first unit of the job within its phase (unit = one element of W)
+  // Phase 1, gated output: the result is silu(G) · (sum + bias), G the gate
+  // job's stored output (same N and blocks), read once gate_fin[b] is set.
+  const void* gate_y;      // null: no gate
+  int64_t gate_ld;
+  int gate_f32;
+  const unsigned int* gate_fin;
+  unsigned int* fin;       // phase 1: [blocks] 1 once the block is written (gates), or null
 };
 
 struct StreamArgs {
@@ -163,6 +170,10 @@ inline int stream_block_cols(int64_t n) {
 }
 
 cudaError_t launch_stream(const StreamArgs& a, int grid, cudaStream_t stream, bool dependent);
+// Y[m, n] = silu(G[m, n]) · P[m, n] for m < M, n < N (G bf16 or fp32 at
+// stride ld_g, P fp32 at stride N, Y bf16 or fp32 at stride ld_y).
+cudaError_t launch_silu_mul(const void* G, int64_t ld_g, bool g_f32, const float* P, void* Y,
+                            int64_t ld_y, bool y_f32, int64_t M, int64_t N, cudaStream_t stream);
 
 // ------------------------------------------------------------------ decode
 // out[m, n] = sum_k V[m, k] · W[k, n] for m < M (M <= 16), W a bf16 [Kd, Nd]

@@ -110,6 +110,30 @@ __device__ __forceinline__ int row_shift(const StreamJob& J, int64_t k, int64_t 
   return static_cast<int>(((reinterpret_cast<uintptr_t>(J.W) >> 1) + k * J.ldw + n0) & 7);
 }
 
+// Wait (bounded) until *flag is set.  One lane waits; the warp follows it.
+__device__ __forceinline__ bool wait_flag(const StreamArgs& a, const unsigned int* flag, int lane) {
+  bool ok = true;
+  if (lane == 0 && ld_acquire_u32(flag) == 0u) {
+    const unsigned long long t_start = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (ld_acquire_u32(flag) != 0u) break;
+      if ((it & 63u) == 0u) {
+        if (aborted(a.wait)) {
+          ok = false;
+          break;
+        }
+        if (global_ns() - t_start > a.wait.timeout_ns) {
+          record_timeout(a.wait, kWhereStreamReady);
+          ok = false;
+          break;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // Wait (bounded) until the blocks of phase-0 job S holding columns
 // [c0, c1] are finished.  One lane waits; the warp follows it.
 __device__ __forceinline__ bool wait_ready(const StreamArgs& a, const StreamJob& S, int64_t c0,
@@ -392,13 +416,25 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
     __syncthreads();
     if (*s_last) {
       // This piece completed the block: write it, re-zero the workspace.
+      // A gated block first waits (bounded) for the gate's same block.
       __threadfence();
+      if (J.gate_y) {
+        if (threadIdx.x < 32) (void)wait_flag(a, J.gate_fin + sg.b, threadIdx.x & 31);
+        __syncthreads();
+      }
       for (int i = threadIdx.x; i < a.M * wb; i += kThreads) {
         const int m = i / wb, c = i - m * wb;
         float* src = J.acc + m * J.ld_acc + n0 + c;
         float v = __ldcg(src);
         __stcg(src, 0.f);
         if (J.bias) v += __bfloat162float(J.bias[n0 + c]);
+        if (J.gate_y) {
+          const int64_t gi = m * J.gate_ld + n0 + c;
+          const float gv = J.gate_f32 ? __ldcg(static_cast<const float*>(J.gate_y) + gi)
+                                      : __bfloat162float(__ushort_as_bfloat16(__ldcg(
+                                            static_cast<const unsigned short*>(J.gate_y) + gi)));
+          v *= gv / (1.f + expf(-gv));
+        }
         if (J.out_f32)
           J.out_f32[m * J.ld_out + n0 + c] = v;
         else
@@ -410,15 +446,20 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
         J.cnt[sg.b] = 0u;
         if (J.phase == 0) {
           st_release_u32(J.ready + sg.b, 1u);
-        } else if (atomicAdd(a.done, 1u) + 1u == static_cast<unsigned int>(a.n_final)) {
-          // Every phase-1 block is finished, so every read of a phase-0
-          // result is done: clear the flags for the next launch.
-          for (int j = 0; j < a.n_jobs; ++j)
-            if (a.job[j].phase == 0) {
-              const int nb = (a.job[j].N + a.job[j].cb - 1) / a.job[j].cb;
-              for (int b = 0; b < nb; ++b) a.job[j].ready[b] = 0u;
+        } else {
+          if (J.fin) st_release_u32(J.fin + sg.b, 1u);
+          if (atomicAdd(a.done, 1u) + 1u == static_cast<unsigned int>(a.n_final)) {
+            // Every phase-1 block is finished, so every read of a flag is
+            // done: clear them for the next launch.
+            for (int j = 0; j < a.n_jobs; ++j) {
+              const StreamJob& Q = a.job[j];
+              const int nb = (Q.N + Q.cb - 1) / Q.cb;
+              unsigned int* f = Q.phase == 0 ? Q.ready : Q.fin;
+              if (f)
+                for (int b = 0; b < nb; ++b) f[b] = 0u;
             }
-          *a.done = 0u;
+            *a.done = 0u;
+          }
         }
       }
     }
@@ -445,6 +486,34 @@ cudaError_t launch_mt(const StreamArgs& a, int grid, cudaStream_t stream, bool d
 }
 
 }  // namespace
+
+namespace {
+__global__ void silu_mul_kernel(const void* G, int64_t ld_g, int g_f32, const float* P, void* Y,
+                                int64_t ld_y, int y_f32, int64_t M, int64_t N) {
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, n = i - m * N;
+    const float g = g_f32 ? static_cast<const float*>(G)[m * ld_g + n]
+                          : __bfloat162float(static_cast<const __nv_bfloat16*>(G)[m * ld_g + n]);
+    const float v = P[i] * (g / (1.f + expf(-g)));
+    if (y_f32)
+      static_cast<float*>(Y)[m * ld_y + n] = v;
+    else
+      static_cast<__nv_bfloat16*>(Y)[m * ld_y + n] = __float2bfloat16_rn(v);
+  }
+}
+}  // namespace
+
+cudaError_t launch_silu_mul(const void* G, int64_t ld_g, bool g_f32, const float* P, void* Y,
+                            int64_t ld_y, bool y_f32, int64_t M, int64_t N, cudaStream_t stream) {
+  const int64_t total = M * N;
+  if (total == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148 * 8);
+  silu_mul_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(G, ld_g, g_f32 ? 1 : 0, P, Y,
+                                                                     ld_y, y_f32 ? 1 : 0, M, N);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_stream(const StreamArgs& a, int grid, cudaStream_t stream, bool dependent) {
   if (a.M > 8) return cudaErrorInvalidValue;

@@ -84,6 +84,25 @@ def test_packed_halves_are_accepted_by_validation(L):
     assert L.lr_linear_group(arr, 2, 3, None) == lr.LR_ERR_INVALID_ARG
 
 
+def test_silu_gate_validation(L):
+    """A gate must be another projection of the group, with the same N and
+    no gate of its own; checked before anything reaches the device."""
+    def group(gates, ns=(16, 16, 16)):
+        arr = (lr.LrProj * len(ns))()
+        for i, (n, g) in enumerate(zip(ns, gates)):
+            arr[i] = lr.LrProj(0x100000, 8, 0x200000 + i * 0x10000, 0x300000 + i * 0x10000, None,
+                               0x4000000 + i * 0x100000, n, 4, n, 0, g)
+        return L.lr_linear_group(arr, len(ns), 3, None)
+    for bad in [(0, 4, 0),      # gate index past the group
+                (0, 2, 0),      # its own gate
+                (2, 1, 0),      # the gate has a gate
+                (0, -1, 0)]:    # negative
+        assert group(bad) == lr.LR_ERR_INVALID_ARG, bad
+    assert group((0, 1, 0), ns=(16, 24, 16)) == lr.LR_ERR_INVALID_ARG  # N differs
+    # A valid group gets past validation (then needs a device).
+    assert group((0, 1, 0)) != lr.LR_ERR_INVALID_ARG
+
+
 def test_controls(L):
     assert L.lr_set_path(7) == lr.LR_ERR_INVALID_ARG
     assert L.lr_set_path(0) == lr.LR_OK
