@@ -49,7 +49,7 @@ DECODE_SHAPES = [("gate_up", 4096, 2867, 14336), ("down", 14336, 2867, 4096)]
 
 # B200 nominal figures (dense bf16 tensor throughput, HBM3e bandwidth of the
 # HGX part): the denominators of `frac_spec`.  The targets (70% prefill, 80%
-# decode) are judged on the measured peaks (`frac`); `frac_spec` is reported
+# decode) are stated against the measured peaks (`frac`); `frac_spec` is reported
 # beside them.
 SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 7700.0,
               "source": "B200 nominal: 2.25 PFLOP/s dense bf16, 7.7 TB/s HBM3e"}
@@ -753,6 +753,8 @@ def main():
     ap.add_argument("--gac-sweep", action="store_true",
                     help="only time lr_linear at the ranks the GAC planner sweeps, per weight shape")
     ap.add_argument("--gac-m", type=int, default=2048, help="tokens for --gac-sweep")
+    ap.add_argument("--profile-layer", action="store_true",
+                    help="only the decoder layer at M = 1 through lr_linear_group (for ncu captures)")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="M",
                     help="only decode steps of the gate/up shape at this M (for ncu captures)")
     args = ap.parse_args()
@@ -764,6 +766,8 @@ def main():
         return run_sweep()
     if args.profile_decode:
         return run_profile_decode(args)
+    if args.profile_layer:
+        return run_profile_layer(args)
     if args.gac_sweep:
         return run_gac_sweep(args)
     return run_ours(args)
@@ -791,6 +795,39 @@ def run_profile_decode(args):
     torch.cuda.synchronize()
     status = lr.last_device_status()
     print(json.dumps({"profile_run": "decode", "M": dm, "K": dk, "r": dr, "N": dn,
+                      "gpu_launches": int(lr.kernel_launch_count() - launches0),
+                      "status": int(status)}))
+    return 0 if status == lr.LR_OK else 1
+
+
+def run_profile_layer(args):
+    """The Llama-3-8B decoder layer at M = 1 through lr_linear_group (one
+    streamed launch per call; seed 7, N_int 14336), warmup + steps calls,
+    for ncu captures of this command; no timing line."""
+    import torch
+    import rank_linear_layers_b200 as lr
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_int = 14336
+    layer = lrgen.decoder_layer(1, seed=7, n_int=n_int)
+    xs = {k: _dev_bits(v, dev) for k, v in layer["inputs"].items()}
+    packed = torch.empty((1, 2 * n_int), dtype=torch.bfloat16, device=dev)
+    entries = []
+    for name, p in layer["projs"].items():
+        e = dict(X=xs[p["x"]], A=_dev_bits(p["A"], dev), B=_dev_bits(p["B"], dev), K=p["K"],
+                 r=p["r"], N=p["N"])
+        if name in ("gate", "up"):
+            e["Y_ptr"] = packed.data_ptr() + (0 if name == "gate" else 2 * n_int)
+            e["ld_y"] = 2 * n_int
+        else:
+            e["Y"] = torch.empty((1, p["N"]), dtype=torch.bfloat16, device=dev)
+        entries.append(e)
+    launches0 = lr.kernel_launch_count()
+    for _ in range(args.warmup + args.steps):
+        lr.lr_linear_group(entries, 1)
+    torch.cuda.synchronize()
+    status = lr.last_device_status()
+    print(json.dumps({"profile_run": "layer", "M": 1, "ranks": layer["ranks"],
                       "gpu_launches": int(lr.kernel_launch_count() - launches0),
                       "status": int(status)}))
     return 0 if status == lr.LR_OK else 1
