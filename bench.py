@@ -120,6 +120,15 @@ def prefill_inputs():
     return p
 
 
+def rank_rows(rank, rows=None):
+    """Rank `rank`'s rows of the whole job's batch of X: rows rank·M ..
+    rank·M + M - 1 of one matrix drawn by the prefill generator (X ~ N(0,1),
+    seed 0), the factors replicated on every rank (data parallel, weak
+    scaling: no data-path collective).  `rows` overrides M (tests)."""
+    m = M if rows is None else rows
+    return lrgen.normal_bf16(0, lrgen.TENSOR_ID["X"], (m, K), 1.0, row0=rank * m)
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """SM clock and clock-event reasons sampled every 5 ms through NVML
@@ -527,7 +536,9 @@ def run_ours(args):
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    X0, A0, B0 = to_dev(p["X"]), to_dev(p["A"]), to_dev(p["B"])
+    # This rank's rows of the whole job's batch (rank 0: the cached rows).
+    X0 = to_dev(p["X"] if rank == 0 else rank_rows(rank))
+    A0, B0 = to_dev(p["A"]), to_dev(p["B"])
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     step_bytes = (X0.numel() + A0.numel() + B0.numel()) * 2
     copies = max(2, math.ceil(2 * l2 / step_bytes) + 1)

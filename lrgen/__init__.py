@@ -113,10 +113,17 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
         return u.view(np.float32).astype(np.float64)
 
 
-def normal_bf16(seed: int, tensor_id: int, shape, std: float = 1.0) -> np.ndarray:
-    """bf16 bits of N(0, std²) draws with the given shape (row-major counters)."""
+def normal_bf16(seed: int, tensor_id: int, shape, std: float = 1.0, row0: int = 0) -> np.ndarray:
+    """bf16 bits of N(0, std²) draws with the given shape (row-major counters).
+
+    ``row0``: the rows row0 .. row0 + shape[0] - 1 of a taller matrix with the
+    same columns (its counters start at row0·cols), so that row blocks drawn
+    separately (one per rank of a data-parallel batch) are the matching rows
+    of the matrix drawn whole.
+    """
     n = int(np.prod(shape)) if len(shape) else 1
-    return bf16_bits(normal(seed, tensor_id, n) * std).reshape(shape)
+    cols = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    return bf16_bits(normal(seed, tensor_id, n, start=row0 * cols) * std).reshape(shape)
 
 
 def lowrank_problem(M: int, K: int, r: int, N: int, seed: int = 0,
