@@ -44,10 +44,6 @@ __device__ __forceinline__ uint32_t stage_raw(uint8_t* dst, const void* p, size_
   return static_cast<uint32_t>(reinterpret_cast<uintptr_t>(p) - lo);
 }
 
-__device__ __forceinline__ uint32_t bf_bits(const uint8_t* base, uint32_t off, int64_t idx) {
-  return *reinterpret_cast<const unsigned short*>(base + off + static_cast<uint32_t>(idx) * 2u);
-}
-
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
   asm volatile(
@@ -97,7 +93,9 @@ __host__ __device__ inline TinyLayout tiny_layout(int64_t K, int64_t r, int64_t 
 // (zero-padded to a multiple of 16), W from raw bf16 (wbase + woff, row
 // pitch ldw; entries past depth or cols read as zero).  Warps take
 // (n tile, k range) tasks; the k ranges' partial sums are added in order and
-// handed to store(m, c, value).
+// handed to store(m, c, value), warp m taking row m.  The shared-memory
+// offsets fit in 32 bits (at most 200 KB); a lane's column is checked once
+// per task and the rows once per k step.
 template <typename Store>
 __device__ __forceinline__ void tiny_mma_product(const uint16_t* vh, const uint16_t* vl, int vp,
                                                  const uint8_t* wbase, uint32_t woff, int64_t ldw,
@@ -106,32 +104,45 @@ __device__ __forceinline__ void tiny_mma_product(const uint16_t* vh, const uint1
   const int g = lane >> 2, t = lane & 3;
   const int nt = (cols + 7) / 8, ks = (depth + 15) / 16;
   const int split = tiny_ksplit(nt, ks);
+  const uint32_t row_bytes = static_cast<uint32_t>(ldw) * 2u;
   for (int task = warp; task < nt * split; task += kTinyThreads / 32) {
     const int n_tile = task % nt, sp = task / nt;
     const int k0 = ks * sp / split, k1 = ks * (sp + 1) / split;
     const int n = n_tile * 8 + g;
+    const bool n_in = n < cols;
+    // This lane's column of W, and its A-fragment rows of V.
+    const uint8_t* wcol = wbase + woff + 2u * static_cast<uint32_t>(n_in ? n : 0);
+    const uint32_t* vh0 = reinterpret_cast<const uint32_t*>(vh + g * vp) + t;
+    const uint32_t* vh8 = reinterpret_cast<const uint32_t*>(vh + (g + 8) * vp) + t;
+    const uint32_t* vl0 = vl ? reinterpret_cast<const uint32_t*>(vl + g * vp) + t : nullptr;
+    const uint32_t* vl8 = vl ? reinterpret_cast<const uint32_t*>(vl + (g + 8) * vp) + t : nullptr;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     for (int kstep = k0; kstep < k1; ++kstep) {
       const int kb = kstep * 16;
-      auto afrag = [&](const uint16_t* v, uint32_t (&a)[4]) {
-        const uint32_t* r0 = reinterpret_cast<const uint32_t*>(v + g * vp + kb);
-        const uint32_t* r8 = reinterpret_cast<const uint32_t*>(v + (g + 8) * vp + kb);
-        a[0] = r0[t];
-        a[1] = r8[t];
-        a[2] = r0[t + 4];
-        a[3] = r8[t + 4];
-      };
+      const int ka = kb + 2 * t;
       auto w = [&](int k) -> uint32_t {
-        return (k < depth && n < cols) ? bf_bits(wbase, woff, static_cast<int64_t>(k) * ldw + n) : 0u;
+        return (n_in && k < depth)
+                   ? *reinterpret_cast<const unsigned short*>(wcol + static_cast<uint32_t>(k) * row_bytes)
+                   : 0u;
       };
-      const uint32_t b0 = w(kb + 2 * t) | (w(kb + 2 * t + 1) << 16);
-      const uint32_t b1 = w(kb + 2 * t + 8) | (w(kb + 2 * t + 9) << 16);
-      uint32_t a[4];
-      afrag(vh, a);
-      mma16816(d, a, b0, b1);
+      uint32_t b0, b1;
+      if (n_in && kb + 16 <= depth) {
+        const uint8_t* p = wcol + static_cast<uint32_t>(ka) * row_bytes;
+        b0 = *reinterpret_cast<const unsigned short*>(p) |
+             (static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(p + row_bytes)) << 16);
+        const uint8_t* q = p + 8u * row_bytes;
+        b1 = *reinterpret_cast<const unsigned short*>(q) |
+             (static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(q + row_bytes)) << 16);
+      } else {
+        b0 = w(ka) | (w(ka + 1) << 16);
+        b1 = w(ka + 8) | (w(ka + 9) << 16);
+      }
+      const int kw = kb / 2;  // 32-bit words into a V row
+      uint32_t av[4] = {vh0[kw], vh8[kw], vh0[kw + 4], vh8[kw + 4]};
+      mma16816(d, av, b0, b1);
       if (vl) {
-        afrag(vl, a);
-        mma16816(d, a, b0, b1);
+        uint32_t al[4] = {vl0[kw], vl8[kw], vl0[kw + 4], vl8[kw + 4]};
+        mma16816(d, al, b0, b1);
       }
     }
     // C fragment: rows g, g + 8; columns 2t, 2t + 1 of the n tile.
@@ -143,10 +154,12 @@ __device__ __forceinline__ void tiny_mma_product(const uint16_t* vh, const uint1
     pp[(g + 8) * nt * 8 + c + 1] = d[3];
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < 16 * cols; i += kTinyThreads) {
-    const int m = i / cols, c = i - m * cols;
+  // Warp m adds up and stores row m (16 warps, 16 rows).
+  static_assert(kTinyThreads / 32 == 16, "one warp per token row");
+  const int m = warp;
+  for (int c = lane; c < cols; c += 32) {
     float v = 0.f;
-    for (int sp = 0; sp < split; ++sp) v += part[(static_cast<int64_t>(sp) * 16 + m) * nt * 8 + c];
+    for (int sp = 0; sp < split; ++sp) v += part[(sp * 16 + m) * nt * 8 + c];
     store(m, c, v);
   }
   __syncthreads();
@@ -167,25 +180,25 @@ __global__ void __launch_bounds__(kTinyThreads, 1) tiny_layer_kernel(TinyArgs a)
   uint8_t* bs = smem + L.braw;
   const uint32_t ao = stage_raw(as, a.A, static_cast<size_t>(K) * r * 2);
   const uint32_t bo = stage_raw(bs, a.B, static_cast<size_t>(r) * N * 2);
-  // X into aligned bf16 rows while A and B arrive (zero past M and K).
+  // X into aligned bf16 rows while A and B arrive (zero past M and K);
+  // warp m takes row m.
   const unsigned short* X = static_cast<const unsigned short*>(a.X);
-  for (int i = threadIdx.x; i < 16 * L.kp; i += kTinyThreads) {
-    const int m = i / L.kp, k = i - m * L.kp;
-    xs[i] = (m < M && k < K) ? X[static_cast<int64_t>(m) * K + k] : static_cast<unsigned short>(0);
-  }
+  const int wm = threadIdx.x >> 5, wl = threadIdx.x & 31;
+  for (int k = wl; k < L.kp; k += 32)
+    xs[wm * L.kp + k] = (wm < M && k < K) ? X[static_cast<int64_t>(wm) * K + k]
+                                           : static_cast<unsigned short>(0);
   cp_async_wait_all();
   __syncthreads();
   // T = X·A in fp32; then its bf16 hi and lo parts (zero past r) for the
   // second product, so that T keeps about 16 bits.
   tiny_mma_product(xs, nullptr, L.kp, as, ao, r, K, r, part,
                    [&](int m, int c, float v) { tf[m * r + c] = v; });
-  for (int i = threadIdx.x; i < 16 * L.rp; i += kTinyThreads) {
-    const int m = i / L.rp, c = i - m * L.rp;
-    const float v = c < r ? tf[m * r + c] : 0.f;
+  for (int c = wl; c < L.rp; c += 32) {
+    const float v = c < r ? tf[wm * r + c] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-    th[i] = __bfloat16_as_ushort(hi);
-    tl[i] = __bfloat16_as_ushort(lo);
+    th[wm * L.rp + c] = __bfloat16_as_ushort(hi);
+    tl[wm * L.rp + c] = __bfloat16_as_ushort(lo);
   }
   __syncthreads();
   // Y = T·B + bias.
