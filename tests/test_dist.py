@@ -88,3 +88,62 @@ def test_two_rank_row_shards_match_the_whole_batch():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert same_rows and same_out
+
+
+def _rsplit_worker(rank, world, port, q):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import lrgen
+        import oracle
+        from rank_linear_layers_b200 import rsplit
+        M, K, r, N = 5, 96, 73, 40
+        p = lrgen.lowrank_problem(M, K, r, N, seed=11, bias=True)
+        r0, r1 = rsplit.rsplit_bounds(r, world, rank)
+
+        def ref_partial(X, A, B, bias):
+            # The oracle on this rank's slice (fp64 -> fp32), bias as given.
+            return torch.from_numpy(oracle.lr_linear(X, A, B, bias).astype(np.float32))
+
+        Y = rsplit.lr_linear_rsplit(p["X"], np.ascontiguousarray(p["A"][:, r0:r1]),
+                                    np.ascontiguousarray(p["B"][r0:r1, :]), p["bias"],
+                                    local_product=ref_partial)
+        whole = oracle.lr_linear(p["X"], p["A"], p["B"], p["bias"])
+        err = float(np.max(np.abs(Y.numpy().astype(np.float64) - whole)))
+        q.put((rank, r0, r1, err, float(np.sqrt(np.mean(whole ** 2)))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_rsplit_sums_the_slices():
+    """r split over 2 gloo ranks: each rank's slice of A and B (16-aligned
+    bounds), one all-reduce; every rank ends with the whole layer's output
+    (bias added once), up to the fp32 rounding of the partials."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rsplit_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (_, a0, a1, e0, rms), (_, b0, b1, e1, _) = out
+    assert (a0, a1, b0, b1) == (0, 32, 32, 73)  # five 16-wide pieces: 2 + 3
+    assert max(e0, e1) <= 1e-6 * rms
+
+
+def test_rsplit_bounds():
+    from rank_linear_layers_b200.rsplit import rsplit_bounds
+    for r in (0, 1, 15, 16, 17, 1741, 2867, 4096):
+        for world in (1, 2, 3, 4, 8):
+            spans = [rsplit_bounds(r, world, i) for i in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == r
+            for (x0, x1), (y0, y1) in zip(spans, spans[1:]):
+                assert x1 == y0 and x0 <= x1
+            assert all(x0 % 16 == 0 for x0, _ in spans)
