@@ -340,7 +340,8 @@ lr_status lr_gac_select(int n_items, const int* n_cand, const int64_t* cost, con
 /* Counts the kernels launched by this library in this process. */
 int64_t lr_kernel_launch_count(void);
 
-/* Frees every workspace and staging buffer (synchronises each device). */
+/* Frees every workspace, staging buffer and decode piece table
+ * (synchronises each stream the library used). */
 lr_status lr_release_workspaces(void);
 
 #ifdef __cplusplus

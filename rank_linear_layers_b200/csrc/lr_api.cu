@@ -397,7 +397,7 @@ void stream_add_pair(StreamArgs& a, const StreamPair& p, char** zero, char** scr
 // Every CTA's pieces for a set of job shapes, computed once on the host and
 // kept on the device (a few KB per set of shapes; the kernel reads its own
 // instead of computing them, which took its threads microseconds).  Kept
-// for the life of the process; a decode loop uses a handful of shapes.
+// until lr_release_workspaces; a decode loop uses a handful of shapes.
 struct PieceTable {
   StreamSeg* pieces = nullptr;
   int* off = nullptr;
@@ -1670,16 +1670,30 @@ lr_status lr_release_workspaces(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_ws) {
-    if (!kv.second.ptr && !kv.second.ctrs && !kv.second.split_ws && !kv.second.rp_area[0]) continue;
+    if (!kv.second.ptr && !kv.second.ctrs && !kv.second.split_ws && !kv.second.rp_area[0] &&
+        !kv.second.act)
+      continue;
     cudaSetDevice(kv.first.first);
     cudaStreamSynchronize(kv.first.second);
     if (kv.second.ptr) cudaFree(kv.second.ptr);
     if (kv.second.ctrs) cudaFree(kv.second.ctrs);
     if (kv.second.split_ws) cudaFree(kv.second.split_ws);
+    if (kv.second.act) cudaFree(kv.second.act);
     for (char* a : kv.second.rp_area)
       if (a) cudaFree(a);
   }
   g_ws.clear();
+  {
+    // Every stream that ran the streamed kernel has a workspace, synchronised
+    // above: no launch still reads a piece table.
+    std::lock_guard<std::mutex> plk(g_piece_mu);
+    for (auto& kv : g_piece_tables) {
+      cudaSetDevice(static_cast<int>(kv.first[0]));
+      cudaFree(kv.second.pieces);
+      cudaFree(kv.second.off);
+    }
+    g_piece_tables.clear();
+  }
   g_streams.clear();
   for (auto& kv : g_stage) {
     if (!kv.second.ptr) continue;
