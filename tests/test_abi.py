@@ -157,3 +157,28 @@ def test_header_is_plain_c_and_links(L, tmp_path):
                     "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-llrlinear",
                     f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_lr_proj_layout_matches_the_binding(tmp_path):
+    """The binding's ctypes lr_proj has the C struct's size and field offsets
+    (a mismatch would pass the wrong silu_gate or y_f32 silently)."""
+    import ctypes
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    fields = [name for name, _ in lr.LrProj._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "lr_linear.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu", sizeof(lr_proj));\n'
+        + "".join(f'  printf(" %zu", offsetof(lr_proj, {f}));\n' for f in fields)
+        + '  printf("\\n");\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    want = [ctypes.sizeof(lr.LrProj)] + [getattr(lr.LrProj, f).offset for f in fields]
+    assert got == want
