@@ -66,9 +66,12 @@ typedef enum {
  * Sizes: 0 <= M, K, r, N < 2^31.  M == 0 or N == 0: nothing is launched.
  * K == 0 or r == 0: the sum is empty and Y = bias (or 0).
  *
- * Path: M <= 16 takes the decode kernels (bandwidth-bound streaming of A then
- * B, T kept in fp32; two launches, the second streaming B while the first
- * finishes).  Larger M takes the tcgen05 prefill path: one launch
+ * Path: a layer small enough for one SM (M <= 16; K, r, N <= 4096; X, A, B
+ * and the intermediates within 200 KB of shared memory; contiguous operands;
+ * automatic path only) runs in one CTA and one launch.  Otherwise M <= 16
+ * takes the decode kernels (bandwidth-bound streaming of A then B, T kept in
+ * fp32; two launches, the second streaming B while the first finishes).
+ * Larger M takes the tcgen05 prefill path: one launch
  * computes T = X·A (written once as bf16) and Y = T·B, GEMM2's tiles
  * waiting for GEMM1's rows inside the launch.  Neither path pads r on the
  * host.  Prefill operands whose rows do not start on 32-byte boundaries
