@@ -217,6 +217,18 @@ def factor_pitch(cols: int) -> int:
     return int(lib().lr_factor_pitch(int(cols)))
 
 
+def prepare_factor(W):
+    """A copy of the 2-D factor W stored at row pitch factor_pitch(cols) (a
+    one-time copy when weights are loaded, not a step of a call), returned as
+    the [rows, cols] view to pass to lr_linear_strided: its rows are read in
+    place by every call, with no realignment copy."""
+    import torch
+    rows, cols = W.shape
+    buf = torch.zeros((rows, factor_pitch(cols)), dtype=W.dtype, device=W.device)
+    buf[:, :cols].copy_(W)
+    return buf[:, :cols]
+
+
 def lr_dense(X, W, bias=None, Y=None, stream=None):
     """Y = X·W + bias with the same kernels (the dense comparison)."""
     import torch

@@ -182,3 +182,16 @@ def test_lr_proj_layout_matches_the_binding(tmp_path):
                                           check=True).stdout.split()]
     want = [ctypes.sizeof(lr.LrProj)] + [getattr(lr.LrProj, f).offset for f in fields]
     assert got == want
+
+
+def test_prepare_factor_layout():
+    """prepare_factor: the same values, rows at the library's factor pitch
+    (columns rounded up to 64), unit column stride (host code and the
+    library's pitch rule; no GPU)."""
+    import torch
+    for rows, cols in [(5, 107), (3, 64), (2, 1), (4, 1741)]:
+        W = torch.randn(rows, cols).bfloat16()
+        V = lr.prepare_factor(W)
+        assert tuple(V.shape) == (rows, cols) and V.stride(1) == 1
+        assert V.stride(0) == lr.factor_pitch(cols) == -(-cols // 64) * 64
+        assert torch.equal(V, W)
