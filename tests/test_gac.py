@@ -258,3 +258,30 @@ def test_c_solver_largest_candidate_index(L):
         got = lr.gac_select(costs, scores, bases, budget, 1)
         assert got[0] == want[0] and got[1] == want[1]
     assert lr.gac_select(costs, scores, bases, 10 ** 6, 1)[0] == [254, 1]
+
+
+def test_plan_with_the_measured_b200_sweep():
+    """The committed B200 dimension sweep (`bench.py --gac-sweep`, M = 2048,
+    every rank the 32-layer plan may choose for its four weight shapes) as
+    the planner's cliff filter: the documented outcome (140 candidate ranks
+    dropped, every chosen rank a multiple of 8, the plan's objective
+    unchanged by the filter) holds on the stored data."""
+    import json
+    import os
+    from rank_linear_layers_b200 import gac
+    import lrgen
+    path = os.path.join(os.path.dirname(gac.__file__), "gac_sweep_b200.json")
+    with open(path) as f:
+        sweep = json.load(f)
+    assert sweep["M"] == 2048 and sweep["status"] == 0
+    ws = [gac.Weight(**d) for d in lrgen.gac_model(32, 11)]
+    wt = gac.times_by_weight(ws, sweep["times_us"])
+    cliffs = 0
+    for w in ws:
+        swept = gac.sweep_ranks(w.r_star, limit=min(w.K, w.N))
+        cliffs += len(swept) - len(gac.drop_cliffs(swept, wt.get(w.name, {}), 0.05))
+    assert cliffs == 140
+    measured = gac.plan(ws, times=wt)
+    plain = gac.plan(ws)
+    assert measured.aligned_fraction == 1.0
+    assert measured.objective == plain.objective
