@@ -116,3 +116,14 @@ def test_prefill_svd_construction_eckart_young():
     expect = math.sqrt(head / N)
     assert abs(expect - 0.0443) < 1e-4
     assert abs(float(np.sqrt(np.mean(Y ** 2))) / expect - 1) < 0.06
+
+
+def test_row_blocks_are_rows_of_the_whole():
+    """normal_bf16(..., row0=k): rows k .. k + rows - 1 of the matrix drawn
+    whole (counter-based: any row block can be drawn on its own)."""
+    import numpy as np
+    import lrgen
+    whole = lrgen.normal_bf16(3, 7, (11, 13), 0.5)
+    parts = [lrgen.normal_bf16(3, 7, (n, 13), 0.5, row0=k) for k, n in [(0, 4), (4, 1), (5, 6)]]
+    assert np.array_equal(np.concatenate(parts), whole)
+    assert not np.array_equal(lrgen.normal_bf16(3, 7, (4, 13), 0.5, row0=1), whole[:4])
